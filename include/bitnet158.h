@@ -1,0 +1,187 @@
+/*
+ * bitnet158.h -- C ABI of the B200 (sm_100a) BitLinear forward of BitNet b1.58
+ * (W1.58A8: ternary weights, 8-bit activations).
+ *
+ * The operation (sources are web pages on BitNet b1.58, cited by title and
+ * section):
+ *
+ *   weights     gamma = mean |W| over the whole [N, K] matrix;
+ *               Q(w)  = round(clamp(w / gamma, -1, 1)) in {-1, 0, +1};
+ *               stored as the 2-bit value {0 -> 0, +1 -> 1, -1 -> 2}.
+ *               ("Microsoft BitNet 深度研究报告", 技术原理 item 2, AbsMean 量化)
+ *               Four 2-bit values per byte.  (Write-up of the BitNet b1.58
+ *               2B4T technical report, "GPU端：CUDA内核的定制魔法".)
+ *   activations per token m: s_m = 127 / max_k |x_mk|;
+ *               xq = clamp(round(x * s_m), -127, 127) as int8.
+ *               (BitNet b1.58 2B4T model card, 模型详情 -> 量化: per-token
+ *               absmax 8-bit activations.)
+ *   product     acc[m][n] = sum_k xq[m][k] * Q(W)[n][k], exact in int32
+ *               (the add/subtract form of item 3 of the research report);
+ *               y[m][n] = (float)acc * (gamma / s_m), then optionally ReLU^2
+ *               (model card, 架构: squared ReLU in the FFN; no bias terms).
+ *
+ * Readings where the pages say nothing (the same in the CPU oracle):
+ *   round = half away from zero; gamma is summed in fp64, each row in k
+ *   order, then the rows in n order, and rounded once to fp32; gamma == 0
+ *   gives all-zero codes; an all-zero activation row gives s = 1 and xq = 0;
+ *   y = (float)acc * (gamma / s) with one fp32 division and one fp32
+ *   multiply; bf16 outputs round to nearest even.
+ *   Packed layout: row-major [N][K/4] bytes.  Inside each group of 16
+ *   consecutive elements of a row one little-endian 32-bit word holds
+ *   element 16g + 4j + i at bits [8i + 2j, 8i + 2j + 2), i, j in 0..3 (so
+ *   byte i of the word holds elements i, i+4, i+8, i+12).  Code 3 is never
+ *   written; packed input containing it gives unspecified results.
+ *
+ * Conventions for every entry point:
+ *   - Every array argument is a DEVICE pointer owned by the caller; the
+ *     library keeps no pointer after the call returns and allocates no
+ *     device memory (scratch comes from the caller's workspace argument).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; gamma and s stay on the device.
+ *   - Arguments are checked on the host before anything is launched; a
+ *     failed check returns an error status and launches nothing.  Errors are
+ *     return codes only: no exception, abort or device trap.
+ *   - Arrays are dense row-major.  X, xq, Y and packed must be 16-byte
+ *     aligned; s and gamma 4-byte aligned; workspaces 256-byte aligned.
+ *   - M == 0 or N == 0 is an empty call that returns BITNET_OK and launches
+ *     nothing.  K must be a positive multiple of 16 (one packed word) and at
+ *     most 2^24 (so |acc| <= 127 * K stays inside int32).
+ *   - A kernel that gives up a bounded wait records BITNET_ERR_TIMEOUT in a
+ *     device status word; bitnet_get_device_status() reads and clears it.
+ */
+#ifndef BITNET158_H
+#define BITNET158_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t (declared here without the CUDA headers). */
+typedef struct CUstream_st *bitnet_stream_t;
+
+typedef enum bitnet_status {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size, aliasing */
+    BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K not a positive multiple of 16, or K > 2^24    */
+    BITNET_ERR_MISALIGNED = 3,        /* a pointer breaks the alignment rule above       */
+    BITNET_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed            */
+    BITNET_ERR_TIMEOUT = 5,           /* a device-side bounded wait gave up              */
+    BITNET_ERR_RANGE = 6,             /* reserved: input outside the numeric contract    */
+    BITNET_ERR_WORKSPACE = 7          /* workspace missing or smaller than required      */
+} bitnet_status;
+
+typedef enum bitnet_dtype {
+    BITNET_F32 = 0,
+    BITNET_BF16 = 1,
+    BITNET_I8 = 2,
+    BITNET_I32 = 3
+} bitnet_dtype;
+
+typedef enum bitnet_epilogue {
+    BITNET_EPI_NONE = 0,
+    BITNET_EPI_RELU2 = 1  /* y = max(y, 0)^2, the FFN activation of the model card */
+} bitnet_epilogue;
+
+/* Flag for bitnet_w158a8_matmul: `packed` and `gamma` are not written by the
+ * kernel that precedes this call on `stream`.  With it the kernel may start
+ * streaming the weights from HBM before the preceding kernel has finished
+ * (programmatic dependent launch); the activations are still read, and Y
+ * written, only after the preceding kernel has completed.  Without it the
+ * weights are also read only after that point. */
+#define BITNET_FLAG_WEIGHTS_STATIC 1u
+
+/* ----------------------------------------------------------------------
+ * Weight quantisation: absmean ternary codes, packed four per byte.
+ * ("Microsoft BitNet 深度研究报告", 技术原理 item 2; 2B4T report write-up,
+ * GPU kernel section.)
+ *
+ *   W        [N][K] fp32 or bf16 (w_dtype = BITNET_F32 | BITNET_BF16), finite.
+ *   packed   [N][K/4] bytes, written (layout above).
+ *   gamma    one fp32, written: mean |W| (fp64 sum in the fixed order above).
+ *   workspace at least bitnet_quantize_weights_workspace_size(N, K) bytes of
+ *            device scratch (fp64 row sums); contents on entry don't matter.
+ * N must be positive (the mean of an empty matrix is undefined).
+ * ---------------------------------------------------------------------- */
+size_t bitnet_quantize_weights_workspace_size(int64_t N, int64_t K);
+
+bitnet_status bitnet_quantize_weights(const void *W, bitnet_dtype w_dtype, int64_t N, int64_t K,
+                                      uint8_t *packed, float *gamma, void *workspace,
+                                      size_t workspace_bytes, bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
+ * Per-token absmax activation quantisation.  (Model card of BitNet b1.58
+ * 2B4T, 模型详情 -> 量化.)
+ *
+ *   X    [M][K] fp32 or bf16 (x_dtype), finite.
+ *   xq   [M][K] int8, written: clamp(round_half_away(x * s_m), -127, 127).
+ *   s    [M] fp32, written: 127 / max_k |x_mk| (fp32 division); 1 for an
+ *        all-zero row.
+ * K here may be any positive value up to 2^24 that keeps the rows 16-byte
+ * aligned (K % 16 == 0 for int8 rows).
+ * ---------------------------------------------------------------------- */
+bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K,
+                                  int8_t *xq, float *s, bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
+ * The W1.58A8 BitLinear product y = Q(W) applied to x, with the rescale by
+ * gamma / s and the optional ReLU^2.  (Research report 技术原理 items 2-3;
+ * model card 模型详情; 2B4T report write-up, GPU kernel section.)
+ *
+ *   X        x_dtype = BITNET_F32 | BITNET_BF16: [M][K] raw activations; the
+ *            per-token quantisation runs inside the call (bit-identical to
+ *            bitnet_quantize_act) and `s` must be NULL.
+ *            x_dtype = BITNET_I8: [M][K] xq from bitnet_quantize_act, and `s`
+ *            its [M] scales.
+ *   packed, gamma  from bitnet_quantize_weights for the [N][K] weight.
+ *   epi      BITNET_EPI_NONE or BITNET_EPI_RELU2.
+ *   Y        [M][N], y_dtype = BITNET_F32 | BITNET_BF16, or BITNET_I32 for
+ *            the raw int32 accumulators (epi must then be NONE; the scale is
+ *            not applied).  Y must not overlap X.
+ *   workspace at least bitnet_w158a8_matmul_workspace_size(M, N, K, x_dtype)
+ *            bytes (may be NULL when that is 0).  Contents on entry don't
+ *            matter; the call may overwrite all of it.
+ *   flags    0 or BITNET_FLAG_WEIGHTS_STATIC.
+ * Decode-sized calls (M <= 32) run one fused kernel; larger M runs the
+ * activation quantiser into the workspace and then the tensor-core kernel.
+ * ---------------------------------------------------------------------- */
+size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype);
+
+bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
+                                   const uint8_t *packed, const float *gamma, int64_t M,
+                                   int64_t N, int64_t K, bitnet_epilogue epi, void *Y,
+                                   bitnet_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                                   uint32_t flags, bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
+ * Weightless per-token RMS normalisation, y = x / sqrt(mean_k(x^2) + 1e-6),
+ * fp32 arithmetic, bf16 or fp32 in and out.  Glue between chained
+ * BitLinears: the model card names "subln" normalisation (模型详情 -> 架构)
+ * without a formula, and this is the plain stand-in used by the decode
+ * chain.  Not part of the bit-exact BitLinear contract.
+ *   X [M][K] (x_dtype F32 | BF16), Y [M][K] (y_dtype F32 | BF16); may alias.
+ * ---------------------------------------------------------------------- */
+bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K, void *Y,
+                              bitnet_dtype y_dtype, bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
+ * Status and diagnostics.
+ * ---------------------------------------------------------------------- */
+/* Static English text for a status code (never NULL). */
+const char *bitnet_status_string(bitnet_status status);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: BITNET_OK, or the first error a kernel recorded
+ * (BITNET_ERR_TIMEOUT after a bounded wait gave up). */
+bitnet_status bitnet_get_device_status(bitnet_stream_t stream);
+
+/* ABI version of this header: major * 10000 + minor * 100 + patch. */
+int bitnet_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET158_H */

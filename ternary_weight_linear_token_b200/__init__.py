@@ -1,0 +1,198 @@
+"""Thin Python binding of ``libbitnet158.so``, the B200 (sm_100a) C-ABI
+library for the BitNet b1.58 BitLinear forward (W1.58A8).
+
+Argument marshalling only: every function below checks the torch tensors it
+is given (device, dtype, contiguity, shape), passes their device pointers and
+the current CUDA stream to the C entry point of the same name, and raises
+``BitnetError`` on a non-OK status.  All arithmetic runs in the library's
+CUDA kernels; there is no CPU fallback.  Importing this module fails loudly
+if the library has not been built (``python -m
+ternary_weight_linear_token_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+from .build import LIB as LIB_PATH
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m ternary_weight_linear_token_b200.build`"
+        " (the BitLinear forward has no CPU fallback)")
+
+lib = C.CDLL(LIB_PATH)
+
+# ---------------------------------------------------------------- constants
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, \
+    ERR_WORKSPACE = range(8)
+F32, BF16, I8, I32 = 0, 1, 2, 3
+EPI_NONE, EPI_RELU2 = 0, 1
+FLAG_WEIGHTS_STATIC = 1
+
+_DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.int8: I8, torch.int32: I32}
+
+_P = C.c_void_p
+_I64 = C.c_int64
+_SZ = C.c_size_t
+_ST = C.c_int
+
+_SIGS = {
+    "bitnet_version": ([], C.c_int),
+    "bitnet_status_string": ([_ST], C.c_char_p),
+    "bitnet_get_device_status": ([_P], _ST),
+    "bitnet_quantize_weights_workspace_size": ([_I64, _I64], _SZ),
+    "bitnet_quantize_weights": ([_P, _ST, _I64, _I64, _P, _P, _P, _SZ, _P], _ST),
+    "bitnet_quantize_act": ([_P, _ST, _I64, _I64, _P, _P, _P], _ST),
+    "bitnet_w158a8_matmul_workspace_size": ([_I64, _I64, _I64, _ST], _SZ),
+    "bitnet_w158a8_matmul": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST, _P, _SZ,
+                              C.c_uint32, _P], _ST),
+    "bitnet_rms_norm": ([_P, _ST, _I64, _I64, _P, _ST, _P], _ST),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.bitnet_status_string(status).decode()} (status {status})")
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise BitnetError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtypes=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the BitLinear path has no CPU fallback)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} must have dtype in {dtypes}, got {t.dtype}")
+
+
+def version() -> int:
+    return lib.bitnet_version()
+
+
+def status_string(status: int) -> str:
+    return lib.bitnet_status_string(status).decode()
+
+
+def bitnet_get_device_status(stream=None) -> int:
+    return lib.bitnet_get_device_status(_stream(stream))
+
+
+# ---------------------------------------------------------------- weights
+def bitnet_quantize_weights_workspace_size(N: int, K: int) -> int:
+    return lib.bitnet_quantize_weights_workspace_size(N, K)
+
+
+def bitnet_quantize_weights(W: torch.Tensor, packed: torch.Tensor | None = None,
+                            gamma: torch.Tensor | None = None,
+                            workspace: torch.Tensor | None = None, stream=None):
+    """W [N, K] fp32/bf16 -> (packed [N, K/4] uint8, gamma [1] fp32)."""
+    _dev(W, "W", (torch.float32, torch.bfloat16))
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    need = bitnet_quantize_weights_workspace_size(N, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=W.device)
+    _dev(packed, "packed", (torch.uint8,))
+    _dev(gamma, "gamma", (torch.float32,))
+    st = lib.bitnet_quantize_weights(_ptr(W), _DTYPE[W.dtype], N, K, _ptr(packed), _ptr(gamma),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream))
+    _check(st, "bitnet_quantize_weights")
+    return packed, gamma
+
+
+# ---------------------------------------------------------------- activations
+def bitnet_quantize_act(X: torch.Tensor, xq: torch.Tensor | None = None,
+                        s: torch.Tensor | None = None, stream=None):
+    """X [M, K] fp32/bf16 -> (xq [M, K] int8, s [M] fp32)."""
+    _dev(X, "X", (torch.float32, torch.bfloat16))
+    M, K = X.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if s is None:
+        s = torch.empty(M, dtype=torch.float32, device=X.device)
+    _dev(xq, "xq", (torch.int8,))
+    _dev(s, "s", (torch.float32,))
+    st = lib.bitnet_quantize_act(_ptr(X), _DTYPE[X.dtype], M, K, _ptr(xq), _ptr(s),
+                                 _stream(stream))
+    _check(st, "bitnet_quantize_act")
+    return xq, s
+
+
+# ---------------------------------------------------------------- matmul
+def bitnet_w158a8_matmul_workspace_size(M: int, N: int, K: int, x_dtype) -> int:
+    xd = _DTYPE[x_dtype] if isinstance(x_dtype, torch.dtype) else int(x_dtype)
+    return lib.bitnet_w158a8_matmul_workspace_size(M, N, K, xd)
+
+
+def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                         s: torch.Tensor | None = None, relu2: bool = False,
+                         out_dtype: torch.dtype = torch.bfloat16, Y: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None, weights_static: bool = False,
+                         stream=None) -> torch.Tensor:
+    """Y = BitLinear(X).  X is fp32/bf16 [M, K] (quantised inside the call) or
+    int8 xq [M, K] with its scales ``s`` [M].  out_dtype fp32/bf16, or int32
+    for the raw accumulators (relu2 must then be False)."""
+    _dev(X, "X", (torch.float32, torch.bfloat16, torch.int8))
+    _dev(packed, "packed", (torch.uint8,))
+    _dev(gamma, "gamma", (torch.float32,))
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError(f"packed has {packed.shape[1]} bytes per row, expected K/4 = {K // 4}")
+    if s is not None:
+        _dev(s, "s", (torch.float32,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _dev(Y, "Y", (torch.float32, torch.bfloat16, torch.int32))
+    need = bitnet_w158a8_matmul_workspace_size(M, N, K, X.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.bitnet_w158a8_matmul(_ptr(X), _DTYPE[X.dtype], _ptr(s), _ptr(packed), _ptr(gamma),
+                                  M, N, K, EPI_RELU2 if relu2 else EPI_NONE, _ptr(Y),
+                                  _DTYPE[Y.dtype], _ptr(workspace), ws_bytes,
+                                  FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
+    _check(st, "bitnet_w158a8_matmul")
+    return Y
+
+
+# ---------------------------------------------------------------- glue
+def bitnet_rms_norm(X: torch.Tensor, Y: torch.Tensor | None = None,
+                    out_dtype: torch.dtype | None = None, stream=None) -> torch.Tensor:
+    """Weightless per-token RMS normalisation (decode-chain glue)."""
+    _dev(X, "X", (torch.float32, torch.bfloat16))
+    M, K = X.shape
+    if Y is None:
+        Y = torch.empty((M, K), dtype=out_dtype or X.dtype, device=X.device)
+    _dev(Y, "Y", (torch.float32, torch.bfloat16))
+    st = lib.bitnet_rms_norm(_ptr(X), _DTYPE[X.dtype], M, K, _ptr(Y), _DTYPE[Y.dtype],
+                             _stream(stream))
+    _check(st, "bitnet_rms_norm")
+    return Y

@@ -1,0 +1,251 @@
+// abi.cu -- the C ABI (include/bitnet158.h): argument checks on the host,
+// choice of kernel path, launches on the caller's stream.
+//
+// Every check runs before any CUDA call, so a rejected call has no side
+// effect and needs no GPU.  Paths of bitnet_w158a8_matmul:
+//   decode   M <= 32, K % 64 == 0, the 16-row weight block fits in shared
+//            memory: one fused kernel (activation quantisation inside).
+//   prefill  otherwise, K % 64 == 0: bitnet_quantize_act into the workspace
+//            (unless xq is given), then the tcgen05 tensor-core kernel.
+//   generic  K % 64 != 0: quantise into the workspace, then the dp4a kernel.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/bitnet158.h"
+#include "internal.h"
+
+namespace bitnet {
+
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = int64_t(1) << 24;
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;
+
+struct DeviceInfo {
+  int *status = nullptr;
+  int num_sms = 0;
+  bool ready = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+bitnet_status device_ctx(bitnet_stream_t stream, LaunchCtx *ctx) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BITNET_ERR_CUDA;
+  DeviceInfo &d = g_dev[dev];
+  if (!d.ready) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!d.ready) {
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return BITNET_ERR_CUDA;
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BITNET_ERR_CUDA;
+      d.status = static_cast<int *>(addr);
+      d.num_sms = sms;
+      d.ready = true;
+    }
+  }
+  ctx->stream = reinterpret_cast<cudaStream_t>(stream);
+  ctx->status = d.status;
+  ctx->num_sms = d.num_sms;
+  ctx->pdl = true;
+  return BITNET_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t elem_size(bitnet_dtype t) {
+  switch (t) {
+    case BITNET_F32: return 4;
+    case BITNET_BF16: return 2;
+    case BITNET_I8: return 1;
+    case BITNET_I32: return 4;
+  }
+  return 0;
+}
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na > 0 && nb > 0 && x < y + nb && y < x + na;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+bitnet_status check_k(int64_t K) {
+  if (K <= 0) return BITNET_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return BITNET_OK;
+}
+
+bitnet_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
+
+// Scratch the matmul needs: int8 xq [M][K] and fp32 s [M] whenever the
+// activation quantiser runs as its own kernel (prefill and generic paths
+// with float input).  Pure arithmetic: no CUDA call.
+size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
+  if (M <= 0 || N <= 0 || K <= 0 || x_dtype == BITNET_I8) return 0;
+  if (decode_supported(M, N, K)) return 0;
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+         align256(4 * static_cast<size_t>(M));
+}
+
+}  // namespace
+}  // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+int bitnet_version(void) { return 10000; }
+
+const char *bitnet_status_string(bitnet_status status) {
+  switch (status) {
+    case BITNET_OK: return "ok";
+    case BITNET_ERR_INVALID_ARG: return "invalid argument";
+    case BITNET_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BITNET_ERR_MISALIGNED: return "misaligned pointer";
+    case BITNET_ERR_CUDA: return "CUDA error";
+    case BITNET_ERR_TIMEOUT: return "device wait timed out";
+    case BITNET_ERR_RANGE: return "input outside the numeric contract";
+    case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+size_t bitnet_quantize_weights_workspace_size(int64_t N, int64_t K) {
+  (void)K;
+  return N > 0 ? align256(8 * static_cast<size_t>(N)) : 0;
+}
+
+bitnet_status bitnet_quantize_weights(const void *W, bitnet_dtype w_dtype, int64_t N, int64_t K,
+                                      uint8_t *packed, float *gamma, void *workspace,
+                                      size_t workspace_bytes, bitnet_stream_t stream) {
+  if (W == nullptr || packed == nullptr || gamma == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (w_dtype != BITNET_F32 && w_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (N <= 0 || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_k(K)) return st;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(gamma, 4)) return BITNET_ERR_MISALIGNED;
+  const size_t need = bitnet_quantize_weights_workspace_size(N, K);
+  if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  if (overlap(W, static_cast<size_t>(N) * K * elem_size(w_dtype), packed,
+              static_cast<size_t>(N) * (K / 4)))
+    return BITNET_ERR_INVALID_ARG;
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  return from_cuda(launch_quantize_weights(W, w_dtype, N, K, packed, gamma,
+                                           static_cast<double *>(workspace), ctx));
+}
+
+bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K,
+                                  int8_t *xq, float *s, bitnet_stream_t stream) {
+  if (X == nullptr || xq == nullptr || s == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (M < 0 || M > kMaxRows) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_k(K)) return st;
+  if (!aligned(X, 16) || !aligned(xq, 16) || !aligned(s, 4)) return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), xq, static_cast<size_t>(M) * K))
+    return BITNET_ERR_INVALID_ARG;
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  return from_cuda(launch_quantize_act(X, x_dtype, M, K, xq, s, ctx));
+}
+
+size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
+  return matmul_workspace(M, N, K, x_dtype);
+}
+
+bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
+                                   const uint8_t *packed, const float *gamma, int64_t M,
+                                   int64_t N, int64_t K, bitnet_epilogue epi, void *Y,
+                                   bitnet_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                                   uint32_t flags, bitnet_stream_t stream) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
+    return BITNET_ERR_INVALID_ARG;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32)
+    return BITNET_ERR_INVALID_ARG;
+  if (epi != BITNET_EPI_NONE && epi != BITNET_EPI_RELU2) return BITNET_ERR_INVALID_ARG;
+  if (y_dtype == BITNET_I32 && epi != BITNET_EPI_NONE) return BITNET_ERR_INVALID_ARG;
+  if ((flags & ~BITNET_FLAG_WEIGHTS_STATIC) != 0) return BITNET_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_k(K)) return st;
+  if (X == nullptr || packed == nullptr || gamma == nullptr || Y == nullptr)
+    return BITNET_ERR_INVALID_ARG;
+  if ((x_dtype == BITNET_I8) != (s != nullptr)) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(gamma, 4) ||
+      (s != nullptr && !aligned(s, 4)))
+    return BITNET_ERR_MISALIGNED;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
+              static_cast<size_t>(M) * N * elem_size(y_dtype)))
+    return BITNET_ERR_INVALID_ARG;
+  const size_t need = matmul_workspace(M, N, K, x_dtype);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  }
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  const bool relu2 = epi == BITNET_EPI_RELU2;
+  const bool wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
+
+  if (decode_supported(M, N, K))
+    return from_cuda(launch_decode(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                   wstatic, ctx));
+
+  const int8_t *xq = static_cast<const int8_t *>(X);
+  const float *sq = s;
+  if (x_dtype != BITNET_I8) {
+    int8_t *wxq = static_cast<int8_t *>(workspace);
+    float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                          align256(static_cast<size_t>(M) * K));
+    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, ctx);
+    if (e != cudaSuccess) return BITNET_ERR_CUDA;
+    xq = wxq;
+    sq = ws;
+  }
+  if (prefill_supported(M, N, K))
+    return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, wstatic, ctx));
+  return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
+}
+
+bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K, void *Y,
+                              bitnet_dtype y_dtype, bitnet_stream_t stream) {
+  if (X == nullptr || Y == nullptr) return BITNET_ERR_INVALID_ARG;
+  if ((x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) ||
+      (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16))
+    return BITNET_ERR_INVALID_ARG;
+  if (M < 0 || M > kMaxRows) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_k(K)) return st;
+  if (!aligned(X, 16) || !aligned(Y, 16)) return BITNET_ERR_MISALIGNED;
+  if (M == 0) return BITNET_OK;
+  if (X != Y && overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
+                        static_cast<size_t>(M) * K * elem_size(y_dtype)))
+    return BITNET_ERR_INVALID_ARG;
+  if (X == Y && x_dtype != y_dtype) return BITNET_ERR_INVALID_ARG;
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  return from_cuda(launch_rms_norm(X, x_dtype, M, K, Y, y_dtype, ctx));
+}
+
+bitnet_status bitnet_get_device_status(bitnet_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  int value = 0;
+  if (cudaMemcpyFromSymbol(&value, g_device_status, sizeof(int)) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (value != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+      return BITNET_ERR_CUDA;
+  }
+  return static_cast<bitnet_status>(value);
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// internal.h -- host-side launchers shared between the C-ABI file and the
+// kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace bitnet {
+
+// Element kinds used by the kernels (mirror bitnet_dtype values).
+enum Kind : int { kF32 = 0, kBF16 = 1, kI8 = 2, kI32 = 3 };
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  int *status;      // device status word of the current device
+  int num_sms;
+  bool pdl;         // launch with programmatic stream serialization
+};
+
+// quant_weights.cu
+cudaError_t launch_quantize_weights(const void *W, int w_kind, int64_t N, int64_t K,
+                                    uint8_t *packed, float *gamma, double *row_sums,
+                                    const LaunchCtx &ctx);
+
+// quant_act.cu
+cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
+                                float *s, const LaunchCtx &ctx);
+cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
+                            const LaunchCtx &ctx);
+
+// gemv_decode.cu: fused decode kernel, M <= 32, K % 64 == 0.
+bool decode_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_decode(const void *X, int x_kind, const float *s, const uint8_t *packed,
+                          const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
+                          void *Y, int y_kind, bool weights_static, const LaunchCtx &ctx);
+
+// gemm_generic.cu: any M, K % 16 == 0, int8 activations already quantised.
+cudaError_t launch_generic(const int8_t *xq, const float *s, const uint8_t *packed,
+                           const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
+                           void *Y, int y_kind, const LaunchCtx &ctx);
+
+// gemm_prefill.cu: tcgen05 tensor-core kernel, K % 64 == 0.
+bool prefill_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
+                           const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
+                           void *Y, int y_kind, bool weights_static, const LaunchCtx &ctx);
+
+// Launch helper: cudaLaunchKernelEx with the PDL attribute when ctx.pdl.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     const LaunchCtx &ctx, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = ctx.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ctx.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace bitnet

@@ -1,0 +1,161 @@
+// quant_act.cu -- per-token absmax int8 activation quantisation (BitNet
+// b1.58 2B4T model card, 模型详情 -> 量化: activations to 8-bit integers with
+// per-token absmax), and the weightless RMS normalisation used as glue
+// between chained BitLinears (the card's "subln", formula not given).
+//
+// One warp per token row, 8 rows per CTA: the row's max |x| is reduced with
+// warp shuffles (max is order-independent, so it is exact), then
+// s = 127 / amax and xq = clamp(round_half_away(x * s), -127, 127).  The
+// second pass re-reads the row, which is still in L1.  16 elements (one
+// 16-byte int8 output chunk) per lane-step; K % 16 == 0.
+#include "common.cuh"
+#include "internal.h"
+
+namespace bitnet {
+namespace {
+
+constexpr int kRowsPerCta = 8;
+
+// Load 16 consecutive activations (16-byte aligned) as fp32.
+template <int KIND>
+__device__ __forceinline__ void load16(const void *X, int64_t idx, float (&v)[16]) {
+  if (KIND == kF32) {
+    const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(X) + idx);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = p[q];
+      v[4 * q + 0] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+  } else {
+    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(X) + idx);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 u = p[q];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        v[8 * q + 2 * h + 0] = __uint_as_float(w[h] << 16);
+        v[8 * q + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const void *X, int64_t M,
+                                                                         int64_t K, int8_t *xq,
+                                                                         float *s) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
+  if (m < M) {
+    const int64_t chunks = K / 16;
+    float amax = 0.0f;
+    for (int64_t c = lane; c < chunks; c += 32) {
+      float v[16];
+      load16<KIND>(X, m * K + 16 * c, v);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    }
+    amax = warp_max(amax);
+    const float sm = act_scale(amax);
+    for (int64_t c = lane; c < chunks; c += 32) {
+      float v[16];
+      load16<KIND>(X, m * K + 16 * c, v);
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          w |= (static_cast<uint32_t>(quant_i8(v[4 * q + b], sm)) & 0xFFu) << (8 * b);
+        o[q] = w;
+      }
+      *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) s[m] = sm;
+  }
+  pdl_launch_dependents();
+}
+
+template <int XK, int YK>
+__global__ void __launch_bounds__(32 * kRowsPerCta) rms_norm_kernel(const void *X, int64_t M,
+                                                                     int64_t K, void *Y) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
+  if (m < M) {
+    const int64_t chunks = K / 16;
+    float ss = 0.0f;
+    for (int64_t c = lane; c < chunks; c += 32) {
+      float v[16];
+      load16<XK>(X, m * K + 16 * c, v);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) ss = __fmaf_rn(v[e], v[e], ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, static_cast<float>(K)),
+                                                           1e-6f)));
+    for (int64_t c = lane; c < chunks; c += 32) {
+      float v[16];
+      load16<XK>(X, m * K + 16 * c, v);
+      if (YK == kF32) {
+        float4 *p = reinterpret_cast<float4 *>(static_cast<float *>(Y) + m * K + 16 * c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          p[q] = make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv,
+                             v[4 * q + 3] * inv);
+      } else {
+        uint32_t o[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * h] * inv, v[2 * h + 1] * inv);
+          o[h] = *reinterpret_cast<const uint32_t *>(&b);
+        }
+        uint4 *p = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(Y) + m * K + 16 * c);
+        p[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        p[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
+  pdl_launch_dependents();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
+                                float *s, const LaunchCtx &ctx) {
+  const dim3 grid(static_cast<unsigned>(ceil_div(M, kRowsPerCta)));
+  const dim3 block(32 * kRowsPerCta);
+  if (x_kind == kF32) return launch_k(quantize_act_kernel<kF32>, grid, block, 0, ctx, X, M, K, xq, s);
+  return launch_k(quantize_act_kernel<kBF16>, grid, block, 0, ctx, X, M, K, xq, s);
+}
+
+cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
+                            const LaunchCtx &ctx) {
+  const dim3 grid(static_cast<unsigned>(ceil_div(M, kRowsPerCta)));
+  const dim3 block(32 * kRowsPerCta);
+  if (x_kind == kF32 && y_kind == kF32)
+    return launch_k(rms_norm_kernel<kF32, kF32>, grid, block, 0, ctx, X, M, K, Y);
+  if (x_kind == kF32)
+    return launch_k(rms_norm_kernel<kF32, kBF16>, grid, block, 0, ctx, X, M, K, Y);
+  if (y_kind == kF32)
+    return launch_k(rms_norm_kernel<kBF16, kF32>, grid, block, 0, ctx, X, M, K, Y);
+  return launch_k(rms_norm_kernel<kBF16, kBF16>, grid, block, 0, ctx, X, M, K, Y);
+}
+
+}  // namespace bitnet

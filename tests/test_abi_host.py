@@ -1,0 +1,123 @@
+"""The C-ABI library on the host, without a GPU: it loads, exports every
+function that include/bitnet158.h declares, and rejects bad arguments with the
+documented status before it would touch the device."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnet158.h")
+
+
+@pytest.fixture(scope="module")
+def tw():
+    from ternary_weight_linear_token_b200 import build
+    build.build()
+    import ternary_weight_linear_token_b200 as tw
+    return tw
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("bitnet_quantize_weights", "bitnet_quantize_act", "bitnet_w158a8_matmul",
+                 "bitnet_status_string", "bitnet_get_device_status"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(tw):
+    for name in declared_functions():
+        assert hasattr(tw.lib, name), name
+
+
+def test_status_strings_and_version(tw):
+    for st in range(8):
+        assert isinstance(tw.status_string(st), str) and tw.status_string(st)
+    assert tw.status_string(99) == "unknown status"
+    assert tw.version() == 10000
+
+
+# Fake, suitably aligned device addresses: the calls below must be rejected by
+# the host checks and never dereference them.
+A = C.c_void_p(0x10000000)
+B = C.c_void_p(0x20000000)
+Cc = C.c_void_p(0x30000000)
+G = C.c_void_p(0x40000000)
+WS = C.c_void_p(0x50000000)
+MIS = C.c_void_p(0x20000004)
+
+
+def mm(tw, X=A, xd=1, s=None, P=B, g=G, M=4, N=8, K=64, epi=0, Y=Cc, yd=1, ws=None, wsb=0,
+       flags=0):
+    return tw.lib.bitnet_w158a8_matmul(X, xd, s, P, g, M, N, K, epi, Y, yd, ws, wsb, flags, None)
+
+
+def test_matmul_rejects_bad_arguments(tw):
+    assert mm(tw, X=None) == tw.ERR_INVALID_ARG
+    assert mm(tw, P=None) == tw.ERR_INVALID_ARG
+    assert mm(tw, g=None) == tw.ERR_INVALID_ARG
+    assert mm(tw, Y=None) == tw.ERR_INVALID_ARG
+    assert mm(tw, xd=3) == tw.ERR_INVALID_ARG            # int32 activations
+    assert mm(tw, yd=2) == tw.ERR_INVALID_ARG            # int8 output
+    assert mm(tw, epi=2) == tw.ERR_INVALID_ARG
+    assert mm(tw, yd=3, epi=1) == tw.ERR_INVALID_ARG     # raw int32 with ReLU^2
+    assert mm(tw, flags=2) == tw.ERR_INVALID_ARG
+    assert mm(tw, M=-1) == tw.ERR_INVALID_ARG
+    assert mm(tw, K=0) == tw.ERR_INVALID_ARG
+    assert mm(tw, K=40) == tw.ERR_UNSUPPORTED_SHAPE      # not a multiple of 16
+    assert mm(tw, K=(1 << 24) + 16) == tw.ERR_UNSUPPORTED_SHAPE
+    assert mm(tw, xd=2) == tw.ERR_INVALID_ARG            # int8 input needs s
+    assert mm(tw, s=G) == tw.ERR_INVALID_ARG             # float input takes no s
+    assert mm(tw, X=MIS) == tw.ERR_MISALIGNED
+    assert mm(tw, Y=C.c_void_p(0x30000008)) == tw.ERR_MISALIGNED
+    assert mm(tw, g=C.c_void_p(0x40000002)) == tw.ERR_MISALIGNED
+    # Y overlapping X
+    assert mm(tw, Y=C.c_void_p(0x10000010)) == tw.ERR_INVALID_ARG
+    # prefill-sized float input needs the quantisation workspace
+    assert mm(tw, M=4096, N=6912, K=2560) == tw.ERR_WORKSPACE
+    need = tw.lib.bitnet_w158a8_matmul_workspace_size(4096, 6912, 2560, tw.BF16)
+    assert mm(tw, M=4096, N=6912, K=2560, ws=WS, wsb=need - 1) == tw.ERR_WORKSPACE
+    assert mm(tw, M=4096, N=6912, K=2560, ws=C.c_void_p(0x50000010), wsb=need) == tw.ERR_MISALIGNED
+    # empty calls succeed without touching the device
+    assert mm(tw, M=0) == tw.OK
+    assert mm(tw, N=0) == tw.OK
+
+
+def test_workspace_sizes(tw):
+    f = tw.lib.bitnet_w158a8_matmul_workspace_size
+    assert f(1, 2560, 2560, tw.BF16) == 0          # decode: fused, no scratch
+    assert f(32, 2560, 6912, tw.BF16) == 0
+    assert f(4096, 6912, 2560, tw.I8) == 0          # xq given
+    assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4
+    assert f(5, 64, 48, tw.F32) == 256 + 256        # generic path (K % 64 != 0)
+    assert tw.lib.bitnet_quantize_weights_workspace_size(2560, 2560) == 2560 * 8
+    assert tw.lib.bitnet_quantize_weights_workspace_size(3, 16) == 256
+
+
+def test_quantizers_reject_bad_arguments(tw):
+    q = tw.lib.bitnet_quantize_weights
+    assert q(None, 0, 4, 64, B, G, WS, 256, None) == tw.ERR_INVALID_ARG
+    assert q(A, 2, 4, 64, B, G, WS, 256, None) == tw.ERR_INVALID_ARG      # int8 weights
+    assert q(A, 0, 0, 64, B, G, WS, 256, None) == tw.ERR_INVALID_ARG      # empty matrix
+    assert q(A, 0, 4, 24, B, G, WS, 256, None) == tw.ERR_UNSUPPORTED_SHAPE
+    assert q(A, 0, 4, 64, B, G, None, 0, None) == tw.ERR_WORKSPACE
+    assert q(MIS, 0, 4, 64, B, G, WS, 256, None) == tw.ERR_MISALIGNED
+    a = tw.lib.bitnet_quantize_act
+    assert a(A, 0, 4, 64, None, G, None) == tw.ERR_INVALID_ARG
+    assert a(A, 3, 4, 64, B, G, None) == tw.ERR_INVALID_ARG
+    assert a(A, 0, 4, 20, B, G, None) == tw.ERR_UNSUPPORTED_SHAPE
+    assert a(A, 0, 4, 64, MIS, G, None) == tw.ERR_MISALIGNED
+    assert a(A, 0, 0, 64, B, G, None) == tw.OK
+    r = tw.lib.bitnet_rms_norm
+    assert r(A, 1, 4, 64, A, 0, None) == tw.ERR_INVALID_ARG             # in place, dtype change
+    assert r(A, 1, 4, 64, C.c_void_p(0x10000010), 1, None) == tw.ERR_INVALID_ARG
+    assert r(A, 1, 0, 64, B, 1, None) == tw.OK

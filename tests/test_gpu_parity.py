@@ -1,0 +1,317 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Integers (packed codes, xq, s, int32 accumulators) must be bit-exact.
+Floating-point outputs: fp32 within 1e-6 relative, bf16 within 1 ulp (the
+tolerances of the benchmark spec); the kernels apply the same operations in
+the same order as the oracle, so exact agreement is also counted and reported.
+
+Sizes span several tiles and ragged tails of every kernel path: the fused
+decode kernel (M <= 32, 16-row blocks, 256-element K units), the tcgen05
+prefill kernel (128 x 256 tiles, 128-byte K stages) and the dp4a generic
+kernel (K % 64 != 0).  The full-size prefill workload is checked on sampled
+rows the oracle computes one by one.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import (DEV, as_x, assert_bf16_within_ulp, assert_f32_close, bf16_bits_of, bf16_t,
+                      f32_t, np_of, quantize_weights_both, x_tensor)
+from oracle import ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tw():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from ternary_weight_linear_token_b200 import build
+    build.build()
+    import ternary_weight_linear_token_b200 as tw
+    return tw
+
+
+def _latent(N, K, seed):
+    return synth.latent_weights(np.random.default_rng(seed), N, K)
+
+
+# --------------------------------------------------------------- weights
+WEIGHT_CASES = {
+    "tiny": lambda: synth.config_inputs("tiny")["W"],
+    "decode": lambda: synth.config_inputs("decode")["W"],
+    "qkv": lambda: synth.config_inputs("sweep", proj=0)["W"],
+    "up": lambda: synth.config_inputs("sweep", proj=2)["W"],
+    "down": lambda: synth.config_inputs("sweep", proj=3)["W"],
+    "ragged_37x48": lambda: _latent(37, 48, 1),
+    "one_row_16": lambda: _latent(1, 16, 2),
+    "rows_129_k_272": lambda: _latent(129, 272, 3),
+    "zeros": lambda: np.zeros((20, 64), dtype=np.float32),
+    "ones": lambda: np.ones((20, 64), dtype=np.float32),
+    "minus_ones": lambda: -np.ones((20, 64), dtype=np.float32),
+}
+
+
+@pytest.mark.parametrize("name", sorted(WEIGHT_CASES))
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_weights_bitexact(tw, name, dtype):
+    W = WEIGHT_CASES[name]()
+    pd, gd, po, go = quantize_weights_both(W, dtype)
+    torch.cuda.synchronize()
+    assert np_of(gd)[0].view(np.uint32) == np.float32(go).view(np.uint32), (np_of(gd)[0], go)
+    assert np.array_equal(np_of(pd), po)
+
+
+def test_quantize_weights_boundaries(tw):
+    """The hand-made boundary rows of the oracle pins, on the GPU."""
+    from pins import _BOUNDARY, _BOUNDARY_075
+    for table in (_BOUNDARY, _BOUNDARY_075):
+        W = np.array([[w for w, _ in table]], dtype=np.float32)
+        pd, gd, po, go = quantize_weights_both(W)
+        assert np.array_equal(np_of(pd), po) and np_of(gd)[0] == go
+
+
+# --------------------------------------------------------------- activations
+def _act_cases():
+    yield "tiny", synth.config_inputs("tiny")["x"], "f32"
+    yield "decode", synth.config_inputs("decode", weights=False)["x"], "bf16"
+    yield "sweep_M32_K6912", synth.config_inputs("sweep", M=32, proj=3, weights=False)["x"], "bf16"
+    yield "prefill_rows", synth.config_inputs("prefill", weights=False)["x"][:200], "bf16"
+    rng = np.random.default_rng(11)
+    x = rng.standard_t(3, (7, 48)).astype(np.float32)
+    x[2] = 0.0
+    yield "ragged_zero_row", x, "f32"
+    ties = np.array([[127.0, 0.5, -0.5, 1.5, 2.5, -2.5, 126.5, -126.5, 64.5, -64.5, 3.5, 0.0,
+                      -0.0, 100.25, 1.0, -127.0],
+                     [254.0, 1.0, 3.0, 5.0, -5.0, -254.0, 253.0, 0.0, 2.0, -1.0, -3.0, 7.0, 9.0,
+                      -11.0, 0.5, 0.25]], dtype=np.float32)
+    yield "ties", ties, "f32"
+    yield "ties_bf16", ties, "bf16"
+
+
+@pytest.mark.parametrize("name,x,dtype", list(_act_cases()), ids=lambda v: v if isinstance(v, str) else "")
+def test_quantize_act_bitexact(tw, name, x, dtype):
+    xd, xexact = as_x(x, dtype)
+    xq, s = tw.bitnet_quantize_act(xd)
+    xq_o, s_o = ref.quantize_act(xexact)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_of(s).view(np.uint32), s_o.view(np.uint32))
+    assert np.array_equal(np_of(xq), xq_o)
+
+
+# --------------------------------------------------------------- matmul
+# (M, N, K): decode shapes (M <= 32, K % 64 == 0), prefill shapes (tcgen05),
+# generic shapes (K % 64 != 0).
+SHAPES = [
+    (1, 272, 320), (2, 275, 320), (3, 17, 64), (5, 100, 6912), (8, 160, 2560), (9, 33, 256),
+    (16, 48, 1024), (17, 31, 192), (24, 64, 2560), (31, 47, 640), (32, 96, 6912),
+    (33, 300, 192), (128, 256, 128), (129, 257, 2624), (300, 600, 2560), (256, 520, 64),
+    (5, 77, 48), (40, 33, 80), (1, 19, 2576), (130, 70, 208),
+]
+
+
+def _run_all_outputs(tw, Xd, sd, packed_d, gamma_d, M, N, K, want_acc, s_o, gamma_o):
+    exact = {}
+    for out_dtype, relu2 in ((torch.int32, False), (torch.float32, False), (torch.float32, True),
+                             (torch.bfloat16, False), (torch.bfloat16, True)):
+        Y = tw.bitnet_w158a8_matmul(Xd, packed_d, gamma_d, s=sd, relu2=relu2, out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        if out_dtype == torch.int32:
+            assert np.array_equal(np_of(Y), want_acc), "int32 accumulators differ"
+            continue
+        y_o = ref.epilogue(want_acc, s_o, gamma_o, relu2)
+        if out_dtype == torch.float32:
+            got = np_of(Y)
+            assert_f32_close(got, y_o, 1e-6)
+            exact[("f32", relu2)] = bool(np.array_equal(got.view(np.uint32), y_o.view(np.uint32)))
+        else:
+            got = bf16_bits_of(Y)
+            want = ref.to_bf16(y_o)
+            assert_bf16_within_ulp(got, want, 1)
+            exact[("bf16", relu2)] = bool(np.array_equal(got, want))
+    return exact
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("xdtype", ["f32", "bf16", "i8"])
+def test_matmul_parity(tw, M, N, K, xdtype):
+    rng = np.random.default_rng(M * 7919 + N * 31 + K)
+    W = synth.latent_weights(rng, N, K)
+    x = rng.standard_t(3, (M, K)).astype(np.float32)
+    packed_d, gamma_d, packed_o, gamma_o = quantize_weights_both(W)
+    assert np.array_equal(np_of(packed_d), packed_o)
+    if xdtype == "i8":
+        xq_o, s_o = ref.quantize_act(x)
+        Xd = torch.from_numpy(xq_o).to(DEV)
+        sd = torch.from_numpy(s_o).to(DEV)
+    else:
+        Xd, xexact = as_x(x, xdtype)
+        sd = None
+        xq_o, s_o = ref.quantize_act(xexact)
+    acc_o = ref.matmul_acc(xq_o, packed_o, N, K)
+    exact = _run_all_outputs(tw, Xd, sd, packed_d, gamma_d, M, N, K, acc_o, s_o, gamma_o)
+    assert all(exact.values()), f"within tolerance but not bit-identical: {exact}"
+
+
+def test_matmul_degenerate(tw):
+    K, N = 256, 48
+    x = np.random.default_rng(5).standard_normal((3, K)).astype(np.float32)
+    x[1] = 0.0  # all-zero token row -> s = 1, y row = 0
+    for path_M in (3, 40):  # decode and prefill paths
+        xm = np.resize(x, (path_M, K)).astype(np.float32)
+        Xd = f32_t(xm)
+        for Wv, label in ((np.zeros((N, K), np.float32), "zero"), (np.ones((N, K), np.float32), "ones")):
+            pd, gd = tw.bitnet_quantize_weights(f32_t(Wv))
+            Y = np_of(tw.bitnet_w158a8_matmul(Xd, pd, gd, out_dtype=torch.float32))
+            if label == "zero":
+                assert not Y.any(), "W = 0 must give y = 0"
+            else:
+                xq, s = ref.quantize_act(xm)
+                want = (xq.astype(np.int64).sum(axis=1).astype(np.float32) *
+                        (np.float32(1.0) / s))[:, None].repeat(N, axis=1)
+                assert np.array_equal(Y, want.astype(np.float32)), "W = +1 must give row sums"
+        # zero activation row gives a zero output row
+        pd, gd = tw.bitnet_quantize_weights(f32_t(synth.latent_weights(np.random.default_rng(1), N, K)))
+        Y = np_of(tw.bitnet_w158a8_matmul(Xd, pd, gd, out_dtype=torch.float32))
+        zero_rows = ~xm.any(axis=1)
+        assert zero_rows.any() and not Y[zero_rows].any()
+    # empty batch: no launch, no error
+    empty = torch.empty((0, K), dtype=torch.bfloat16, device=DEV)
+    Y = tw.bitnet_w158a8_matmul(empty, pd, gd)
+    assert Y.shape == (0, N)
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
+def test_sign_flip_on_gpu(tw):
+    rng = np.random.default_rng(9)
+    W = synth.latent_weights(rng, 300, 2560)
+    x = rng.standard_normal((40, 2560)).astype(np.float32)
+    for M in (4, 40):
+        Xd = f32_t(x[:M])
+        p, g = tw.bitnet_quantize_weights(f32_t(W))
+        pn, gn = tw.bitnet_quantize_weights(f32_t(-W))
+        a = np_of(tw.bitnet_w158a8_matmul(Xd, p, g, out_dtype=torch.int32))
+        b = np_of(tw.bitnet_w158a8_matmul(Xd, pn, gn, out_dtype=torch.int32))
+        c = np_of(tw.bitnet_w158a8_matmul(f32_t(-x[:M]), p, g, out_dtype=torch.int32))
+        assert np.array_equal(b, -a) and np.array_equal(c, -a)
+
+
+def test_workspace_too_small_raises(tw):
+    X = torch.zeros((64, 256), dtype=torch.bfloat16, device=DEV)
+    p, g = tw.bitnet_quantize_weights(torch.ones((32, 256), device=DEV))
+    need = tw.bitnet_w158a8_matmul_workspace_size(64, 32, 256, torch.bfloat16)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(tw.BitnetError) as e:
+        tw.bitnet_w158a8_matmul(X, p, g, workspace=ws)
+    assert e.value.status == tw.ERR_WORKSPACE
+
+
+# --------------------------------------------------------------- workloads at full size
+def test_decode_workload_full(tw):
+    """Decode GEMV, M=1, K=N=2560, bf16 in/out: every output against the oracle,
+    plain, with the static-weights flag, and replayed from a CUDA graph."""
+    d = synth.config_inputs("decode")
+    pd, gd, po, go = quantize_weights_both(d["W"])
+    want = ref.to_bf16(ref.bitlinear(d["x"], po, go, d["N"])["y"])
+    Xd = x_tensor(d)
+    for ws in (False, True):
+        Y = tw.bitnet_w158a8_matmul(Xd, pd, gd, weights_static=ws)
+        assert_bf16_within_ulp(bf16_bits_of(Y), want)
+        assert np.array_equal(bf16_bits_of(Y), want)
+    Y = torch.empty((1, d["N"]), dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        tw.bitnet_w158a8_matmul(Xd, pd, gd, Y=Y, weights_static=True)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    Y.zero_()
+    with torch.cuda.graph(graph):
+        for _ in range(4):
+            tw.bitnet_w158a8_matmul(Xd, pd, gd, Y=Y, weights_static=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits_of(Y), want)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_sweep_workload_full(tw, M):
+    """One decoder layer's four projections at M = 1, 8, 32 (Student-t bf16)."""
+    for proj in range(4):
+        d = synth.config_inputs("sweep", M=M, proj=proj)
+        pd, gd, po, go = quantize_weights_both(d["W"])
+        want = ref.to_bf16(ref.bitlinear(d["x"], po, go, d["N"], relu2=d["relu2"])["y"])
+        Y = tw.bitnet_w158a8_matmul(x_tensor(d), pd, gd, relu2=d["relu2"], weights_static=True)
+        assert np.array_equal(bf16_bits_of(Y), want), (M, proj)
+
+
+def test_prefill_workload_full_size_sampled(tw):
+    """Prefill, M=4096, K=2560, N=6912, bf16: the full launch, checked on
+    sampled token rows (tile edges included) against the oracle."""
+    d = synth.config_inputs("prefill")
+    pd, gd, po, go = quantize_weights_both(d["W"])
+    Xd = x_tensor(d)
+    need = tw.bitnet_w158a8_matmul_workspace_size(4096, 6912, 2560, torch.bfloat16)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    Y = tw.bitnet_w158a8_matmul(Xd, pd, gd, workspace=ws, weights_static=True)
+    Yi = tw.bitnet_w158a8_matmul(Xd, pd, gd, workspace=ws, out_dtype=torch.int32)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 63, 127, 128, 129, 1000, 2047, 2048, 3333, 3967, 3968, 4094, 4095])
+    out = ref.bitlinear(d["x"][rows], po, go, d["N"])
+    assert np.array_equal(np_of(Yi)[rows], out["acc"])
+    want = ref.to_bf16(out["y"])
+    got = bf16_bits_of(Y)[rows]
+    assert_bf16_within_ulp(got, want)
+    assert np.array_equal(got, want)
+    # the quantised activations the prefill path wrote into its workspace
+    xq_ws = np_of(ws[: 4096 * 2560]).view(np.int8).reshape(4096, 2560)
+    assert np.array_equal(xq_ws[rows], out["xq"])
+    # any-size property: a zero weight column block gives zero outputs
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
+def test_chain_link_by_link(tw):
+    """Two layers of the 30-layer decode chain: every projection's GPU output
+    against the oracle fed the GPU's own input to that projection."""
+    from ternary_weight_linear_token_b200.chain import DecodeChain
+    layers = []
+    for layer in range(2):
+        layers.append([(f32_t(synth.layer_weights(layer, p)), synth.PROJECTIONS[p][3])
+                       for p in range(4)])
+    chain = DecodeChain(layers)
+    x0 = synth.config_inputs("chain", weights=False)
+    chain.run(x_tensor(x0))
+    torch.cuda.synchronize()
+    x_in = bf16_bits_of(chain.x_in)
+    for li, (proj, bufs) in enumerate(zip(chain.layers, chain.outs)):
+        inputs = [x_in, bf16_bits_of(bufs[0])[:, :chain.d], bf16_bits_of(bufs[1]),
+                  bf16_bits_of(bufs[2])]
+        for pi in range(4):
+            W = synth.layer_weights(li, pi)
+            po, go = ref.quantize_weights(W)
+            assert np.array_equal(np_of(proj[pi]["packed"]), po)
+            xin = synth.bf16_bits_to_f32(inputs[pi])
+            want = ref.to_bf16(ref.bitlinear(xin, po, go, proj[pi]["N"], relu2=proj[pi]["relu2"])["y"])
+            assert np.array_equal(bf16_bits_of(bufs[pi]), want), (li, pi)
+        norm_in = synth.bf16_bits_to_f32(bf16_bits_of(bufs[3]))
+        assert_bf16_within_ulp(bf16_bits_of(bufs[4]), ref.to_bf16(ref.rms_norm(norm_in)), 1)
+        x_in = bf16_bits_of(bufs[4])
+    # graph replay reproduces the eager run bit for bit
+    eager = bf16_bits_of(chain.outs[-1][4]).copy()
+    chain.capture()
+    chain.graph.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits_of(chain.outs[-1][4]), eager)
+
+
+def test_repeatable(tw):
+    d = synth.config_inputs("sweep", M=8, proj=0)
+    pd, gd = tw.bitnet_quantize_weights(f32_t(d["W"]))
+    a = bf16_bits_of(tw.bitnet_w158a8_matmul(x_tensor(d), pd, gd))
+    b = bf16_bits_of(tw.bitnet_w158a8_matmul(x_tensor(d), pd, gd))
+    assert np.array_equal(a, b)
+    assert tw.bitnet_get_device_status() == tw.OK
