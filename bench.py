@@ -140,6 +140,23 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """Max of a per-rank number over all ranks (every rank calls it)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, units_per_step: float, steps: int, seconds: float,
+                    scale: float) -> float:
+    """Whole-job throughput: every rank processes the same per-step work
+    (replicas), timed as the slowest rank."""
+    return world * units_per_step * steps / seconds * scale
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -381,7 +398,8 @@ def main():
         with torch.cuda.graph(kgraph, stream=stream):
             for i in range(args.steps):
                 w["kernel_step"](i, stream)
-    graph.replay()  # one untimed replay: first-launch costs of the graph
+    with torch.cuda.stream(stream):
+        graph.replay()  # one untimed replay: first-launch costs of the graph
     stream.synchronize()
 
     ev0 = torch.cuda.Event(enable_timing=True)
@@ -391,30 +409,27 @@ def main():
     torch.cuda.synchronize(dev)
     bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
                                 getattr(props, "pci_device_id", 0))
-    with ClockSampler(bus) as clocks:
+    with ClockSampler(bus) as clocks, torch.cuda.stream(stream):
         ev0.record(stream)
-        graph.replay()
+        graph.replay()          # replays on the current stream, i.e. `stream`
         ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * w["units_per_step"] * args.steps / (ms * 1e-3) * w["scale"]
+    ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
+    value = whole_job_value(world, w["units_per_step"], args.steps, ms * 1e-3, w["scale"])
 
     # dominant kernel alone (prefill: the tensor-core kernel without the quantiser)
     kms = ms
     if kgraph is not None:
-        kgraph.replay()
-        stream.synchronize()
-        ev0.record(stream)
-        kgraph.replay()
-        ev1.record(stream)
-        ev1.synchronize()
+        with torch.cuda.stream(stream):
+            kgraph.replay()
+            stream.synchronize()
+            ev0.record(stream)
+            kgraph.replay()
+            ev1.record(stream)
+            ev1.synchronize()
         kms = ev0.elapsed_time(ev1)
     per_launch_s = kms * 1e-3 / args.steps
     pk, src = peaks()
@@ -449,11 +464,8 @@ def main():
                 yh.copy_(w["Y"], non_blocking=True)
                 stream.synchronize()
             dt = time.perf_counter() - t0
-        ev = world * w["units_per_step"] * n / dt * w["scale"]
-        if pg:
-            t = torch.tensor([dt], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ev = world * w["units_per_step"] * n / float(t.item()) * w["scale"]
+        dt = max_over_ranks(dt, pg, dev)
+        ev = whole_job_value(world, w["units_per_step"], n, dt, w["scale"])
         e2e = {"value": ev, "unit": w["unit"], "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": n,
                "note": "pinned host activations copied in, BitLinear via the Python binding of "

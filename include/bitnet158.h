@@ -44,7 +44,7 @@
  *   - Arrays are dense row-major.  X, xq, Y and packed must be 16-byte
  *     aligned; s and gamma 4-byte aligned; workspaces 256-byte aligned.
  *   - M == 0 or N == 0 is an empty call that returns BITNET_OK and launches
- *     nothing.  K must be a positive multiple of 16 (one packed word) and at
+ *     nothing; its array pointers may then be NULL.  K must be a positive multiple of 16 (one packed word) and at
  *     most 2^24 (so |acc| <= 127 * K stays inside int32).
  *   - A kernel that gives up a bounded wait records BITNET_ERR_TIMEOUT in a
  *     device status word; bitnet_get_device_status() reads and clears it.

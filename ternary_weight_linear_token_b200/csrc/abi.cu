@@ -144,17 +144,17 @@ bitnet_status bitnet_quantize_weights(const void *W, bitnet_dtype w_dtype, int64
 
 bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K,
                                   int8_t *xq, float *s, bitnet_stream_t stream) {
-  if (X == nullptr || xq == nullptr || s == nullptr) return BITNET_ERR_INVALID_ARG;
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
   if (M < 0 || M > kMaxRows) return BITNET_ERR_INVALID_ARG;
   if (bitnet_status st = check_k(K)) return st;
+  if (M == 0) return BITNET_OK;  // empty: pointers may be NULL
+  if (X == nullptr || xq == nullptr || s == nullptr) return BITNET_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(xq, 16) || !aligned(s, 4)) return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), xq, static_cast<size_t>(M) * K))
     return BITNET_ERR_INVALID_ARG;
   LaunchCtx ctx;
   if (bitnet_status st = device_ctx(stream, &ctx)) return st;
-  return from_cuda(launch_quantize_act(X, x_dtype, M, K, xq, s, ctx));
+  return from_cuda(launch_quantize_act(X, x_dtype, M, K, xq, s, false, ctx));
 }
 
 size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
@@ -175,13 +175,13 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
   if ((flags & ~BITNET_FLAG_WEIGHTS_STATIC) != 0) return BITNET_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
   if (bitnet_status st = check_k(K)) return st;
+  if (M == 0 || N == 0) return BITNET_OK;  // empty: pointers may be NULL
   if (X == nullptr || packed == nullptr || gamma == nullptr || Y == nullptr)
     return BITNET_ERR_INVALID_ARG;
   if ((x_dtype == BITNET_I8) != (s != nullptr)) return BITNET_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(gamma, 4) ||
       (s != nullptr && !aligned(s, 4)))
     return BITNET_ERR_MISALIGNED;
-  if (M == 0 || N == 0) return BITNET_OK;
   if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
               static_cast<size_t>(M) * N * elem_size(y_dtype)))
     return BITNET_ERR_INVALID_ARG;
@@ -199,32 +199,37 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
     return from_cuda(launch_decode(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                    wstatic, ctx));
 
+  (void)wstatic;  // the prefill and generic kernels read the weights after the wait
+  const bool prefill = prefill_supported(M, N, K);
   const int8_t *xq = static_cast<const int8_t *>(X);
   const float *sq = s;
   if (x_dtype != BITNET_I8) {
+    // The prefill kernel takes its own quantiser's output in the K order of
+    // its fast weight unpack; the generic kernel wants natural order.
     int8_t *wxq = static_cast<int8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                           align256(static_cast<size_t>(M) * K));
-    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, ctx);
+    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill, ctx);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     xq = wxq;
     sq = ws;
   }
-  if (prefill_supported(M, N, K))
-    return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, wstatic, ctx));
+  if (prefill)
+    return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                    x_dtype != BITNET_I8, ctx));
   return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
 }
 
 bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K, void *Y,
                               bitnet_dtype y_dtype, bitnet_stream_t stream) {
-  if (X == nullptr || Y == nullptr) return BITNET_ERR_INVALID_ARG;
   if ((x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) ||
       (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16))
     return BITNET_ERR_INVALID_ARG;
   if (M < 0 || M > kMaxRows) return BITNET_ERR_INVALID_ARG;
   if (bitnet_status st = check_k(K)) return st;
+  if (M == 0) return BITNET_OK;  // empty: pointers may be NULL
+  if (X == nullptr || Y == nullptr) return BITNET_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Y, 16)) return BITNET_ERR_MISALIGNED;
-  if (M == 0) return BITNET_OK;
   if (X != Y && overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
                         static_cast<size_t>(M) * K * elem_size(y_dtype)))
     return BITNET_ERR_INVALID_ARG;

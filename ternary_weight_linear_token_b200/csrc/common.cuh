@@ -208,4 +208,22 @@ __device__ __forceinline__ uint32_t unpack_natural(uint32_t w, int j) {
   return c + h * 0xFDu;                                   // 2 -> 0xFF (-1), no carries
 }
 
+// Four int8 values into one 32-bit word, first value in the lowest byte.
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+// 16 int8 activations of one 16-element group, stored in the order in which
+// the byte-permute unpack produces the weights of the matching packed word:
+// elements {0,8,1,9}, {4,12,5,13}, {2,10,3,11}, {6,14,7,15}.
+__device__ __forceinline__ uint4 pack_permuted(const int (&q)[16]) {
+  uint4 o;
+  o.x = pack4(q[0], q[8], q[1], q[9]);
+  o.y = pack4(q[4], q[12], q[5], q[13]);
+  o.z = pack4(q[2], q[10], q[3], q[11]);
+  o.w = pack4(q[6], q[14], q[7], q[15]);
+  return o;
+}
+
 }  // namespace bitnet

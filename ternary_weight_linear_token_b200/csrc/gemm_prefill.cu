@@ -4,20 +4,25 @@
 // the ternary weights {-1, 0, +1} held as int8 (BitNet b1.58 2B4T model card,
 // 模型详情 -> 量化: W1.58A8; "Microsoft BitNet 深度研究报告", 技术原理 items 2-3).
 //
-// Tile: 128 tokens x 256 output features per CTA, K in 128-byte stages.
-//   warp 0      TMA producer: xq tile [128 x 128 B] with the 128-byte swizzle
-//               and the packed weight tile [256 rows x 32 B] (2 bits per
-//               weight stay packed all the way from HBM into shared memory).
-//   warp 1      allocates 256 TMEM columns; one lane issues 4 MMAs
-//               (M=128, N=256, K=32) per stage and commits them to the
-//               stage's "empty" barrier.
-//   warps 2-9   expand each packed word into 16 int8 weights and store them
-//               as the K-major, 128-byte-swizzled B operand; after the K loop
-//               the same 8 warps read the accumulator (tcgen05.ld), apply
-//               y = acc * (gamma / s_m) and the optional ReLU^2, and store Y.
-// A 3-stage ring of mbarriers (TMA full, expansion full, MMA empty) keeps
-// TMA, expansion and MMA of different stages in flight at once.  Every wait
-// is bounded (see common.cuh).
+// Persistent kernel, one CTA per SM, output tiles of 128 tokens x 256
+// features taken round-robin; K in 128-byte stages.
+//   warp 4      TMA producer: xq tile [128 x 128 B] (128-byte swizzle) and the
+//               packed weight tile [256 rows x 32 B] -- 2 bits per weight all
+//               the way from HBM into shared memory -- into a 6-stage ring.
+//   warps 6-13  expand each packed word into 16 int8 weights, stored as the
+//               K-major 128-byte-swizzled B operand in a 2-stage ring.
+//   warp 5      allocates 512 TMEM columns (two 256-column accumulators); one
+//               lane issues 4 MMAs (M=128, N=256, K=32) per stage and commits
+//               them to the barriers that free the TMA and B stages, and,
+//               after a tile's last stage, to the accumulator-full barrier.
+//   warps 0-3   epilogue: tcgen05.ld of the finished accumulator, y = acc *
+//               (gamma / s_m), optional ReLU^2, store; then release the
+//               accumulator, so tile i's epilogue overlaps tile i+1's MMAs.
+// Expansion: with activations quantised by this library (int8 in a K order
+// permuted inside each 16-element group) a packed word becomes 16 weights by
+// four byte-permute lookups (3 instructions per 4 weights); with int8
+// activations given by the caller (natural K order) it uses the in-order
+// shift/mask/multiply unpack.  Every wait is bounded (see common.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -30,15 +35,22 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int kStages = 3;
+constexpr int kTmaStages = 6;
+constexpr int kBxStages = 2;
+constexpr int kEpiWarps = 4;
 constexpr int kExpWarps = 8;
-constexpr int kThreads = 32 * (2 + kExpWarps);
+constexpr int kWarpTma = 4;
+constexpr int kWarpMma = 5;
+constexpr int kWarpExp0 = 6;
+constexpr int kThreads = 32 * (kEpiWarps + 2 + kExpWarps);
 constexpr int kABytes = BM * BK;
-constexpr int kBxBytes = BN * BK;
 constexpr int kBpBytes = BN * BK / 4;
-constexpr int kStageBytes = kABytes + kBxBytes + kBpBytes;
-constexpr int kTmemCols = 256;
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+constexpr int kTmaStageBytes = kABytes + kBpBytes;
+constexpr int kBxBytes = BN * BK;
+constexpr int kTmemCols = 2 * BN;
+constexpr size_t kSmemBytes =
+    1024 + static_cast<size_t>(kTmaStages) * kTmaStageBytes + kBxStages * kBxBytes + 256;
+constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
 
 // Instruction descriptor: s8 x s8 -> s32, both operands K-major, M=128, N=256.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) |
@@ -50,6 +62,7 @@ struct PrefillParams {
   void *Y;
   int *status;
   int64_t M, N, K;
+  int m_tiles, n_tiles;
 };
 
 template <int YK, bool RELU2>
@@ -64,7 +77,9 @@ __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64
       for (int q = 0; q < 4; ++q)
         reinterpret_cast<uint4 *>(dst)[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     } else {
-      for (int e = 0; e < valid; ++e) dst[e] = static_cast<int>(v[e]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (e < valid) dst[e] = static_cast<int>(v[e]);
     }
   } else if (YK == kF32) {
     float y[16];
@@ -76,7 +91,9 @@ __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64
       for (int q = 0; q < 4; ++q)
         reinterpret_cast<float4 *>(dst)[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
     } else {
-      for (int e = 0; e < valid; ++e) dst[e] = y[e];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (e < valid) dst[e] = y[e];
     }
   } else {
     uint32_t h[8];
@@ -92,131 +109,189 @@ __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64
       reinterpret_cast<uint4 *>(dst)[0] = make_uint4(h[0], h[1], h[2], h[3]);
       reinterpret_cast<uint4 *>(dst)[1] = make_uint4(h[4], h[5], h[6], h[7]);
     } else {
-      const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(h);
-      for (int e = 0; e < valid; ++e) dst[e] = src[e];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (e < valid) {
+          const uint32_t bits = (h[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+          reinterpret_cast<uint16_t *>(dst)[e] = static_cast<uint16_t>(bits);
+        }
     }
   }
 }
 
-template <int YK, bool RELU2>
+// 16 int8 weights of one packed word, in the K order the A operand uses.
+template <bool PERM>
+__device__ __forceinline__ uint4 expand_word(uint32_t w) {
+  if (PERM)
+    return make_uint4(__byte_perm(kTernaryLut, 0u, w & 0x3333u),
+                      __byte_perm(kTernaryLut, 0u, (w >> 2) & 0x3333u),
+                      __byte_perm(kTernaryLut, 0u, (w >> 16) & 0x3333u),
+                      __byte_perm(kTernaryLut, 0u, (w >> 18) & 0x3333u));
+  return make_uint4(unpack_natural(w, 0), unpack_natural(w, 1), unpack_natural(w, 2),
+                    unpack_natural(w, 3));
+}
+
+template <int YK, bool RELU2, bool PERM>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *full_tma = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
-  uint64_t *full_x = full_tma + kStages;
-  uint64_t *empty = full_x + kStages;
-  uint64_t *done = empty + kStages;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
+  uint8_t *tma_ring = smem;
+  uint8_t *bx_ring = smem + kTmaStages * kTmaStageBytes;
+  uint64_t *tma_full = reinterpret_cast<uint64_t *>(bx_ring + kBxStages * kBxBytes);
+  uint64_t *tma_empty = tma_full + kTmaStages;
+  uint64_t *bx_full = tma_empty + kTmaStages;
+  uint64_t *bx_empty = bx_full + kBxStages;
+  uint64_t *acc_full = bx_empty + kBxStages;
+  uint64_t *acc_empty = acc_full + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BM;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
   const int kblocks = static_cast<int>((p.K + BK - 1) / BK);
+  const int tiles = p.m_tiles * p.n_tiles;
 
-  if (warp == 0 && lane == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_tma[s], 1);
-      mbar_init(&full_x[s], kExpWarps);
-      mbar_init(&empty[s], 1);
+  if (warp == kWarpTma && lane == 0) {
+    for (int s = 0; s < kTmaStages; ++s) {
+      mbar_init(&tma_full[s], 1);
+      mbar_init(&tma_empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < kBxStages; ++b) {
+      mbar_init(&bx_full[b], kExpWarps);
+      mbar_init(&bx_empty[b], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], kEpiWarps);
+    }
     fence_barrier_init();
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_d = *tmem_holder;
+  const uint32_t tmem_base = *tmem_holder;
 
   // Everything above overlaps the previous kernel; xq and s are its output.
   pdl_wait();
   pdl_launch_dependents();
 
-  if (warp == 0) {
+  if (warp == kWarpTma) {
     if (lane == 0) {
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int s = kb % kStages, it = kb / kStages;
-        if (kb >= kStages && !mbar_wait(&empty[s], (it - 1) & 1, p.status)) break;
-        uint8_t *stage = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&full_tma[s], kABytes + kBpBytes);
-        tma_load_2d(stage, &tmap_a, kb * BK, static_cast<int32_t>(m0), &full_tma[s]);
-        tma_load_2d(stage + kABytes + kBxBytes, &tmap_b, kb * (BK / 4), static_cast<int32_t>(n0),
-                    &full_tma[s]);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int32_t m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kTmaStages;
+          if (it >= kTmaStages && !mbar_wait(&tma_empty[s], ((it / kTmaStages) - 1) & 1, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t *stage = tma_ring + s * kTmaStageBytes;
+          mbar_arrive_expect_tx(&tma_full[s], kTmaStageBytes);
+          tma_load_2d(stage, &tmap_a, kb * BK, m0, &tma_full[s]);
+          tma_load_2d(stage + kABytes, &tmap_b, kb * (BK / 4), n0, &tma_full[s]);
+        }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     if (lane == 0) {
+      uint32_t it = 0;
       bool ok = true;
-      for (int kb = 0; kb < kblocks && ok; ++kb) {
-        const int s = kb % kStages, it = kb / kStages;
-        ok = mbar_wait(&full_tma[s], it & 1, p.status) && mbar_wait(&full_x[s], it & 1, p.status);
-        if (!ok) break;
+      int tl = 0;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        if (tl >= 2 && !mbar_wait(&acc_empty[acc], ((tl >> 1) - 1) & 1, p.status)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * kStageBytes);
-        const uint32_t b_base = a_base + kABytes;
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % kTmaStages, b = it % kBxStages;
+          ok = mbar_wait(&tma_full[s], (it / kTmaStages) & 1, p.status) &&
+               mbar_wait(&bx_full[b], (it / kBxStages) & 1, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(tma_ring + s * kTmaStageBytes);
+          const uint32_t b_base = smem_u32(bx_ring + b * kBxBytes);
 #pragma unroll
-        for (int kk = 0; kk < BK / 32; ++kk)
-          mma_i8(tmem_d, smem_desc_sw128(a_base + 32 * kk), smem_desc_sw128(b_base + 32 * kk),
-                 kIdesc, (kb | kk) != 0 ? 1u : 0u);
-        mma_commit(&empty[s]);
+          for (int kk = 0; kk < BK / 32; ++kk)
+            mma_i8(d, smem_desc_sw128(a_base + 32 * kk), smem_desc_sw128(b_base + 32 * kk), kIdesc,
+                   (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(&tma_empty[s]);
+          mma_commit(&bx_empty[b]);
+        }
+        mma_commit(&acc_full[acc]);
       }
-      mma_commit(done);
+    }
+  } else if (warp >= kWarpExp0) {
+    // ---- expansion: packed [256 rows x 32 B] -> int8 [256 x 128] K-major SW128
+    const int et = (warp - kWarpExp0) * 32 + lane;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % kTmaStages, b = it % kBxStages;
+        if (!mbar_wait(&tma_full[s], (it / kTmaStages) & 1, p.status) ||
+            (it >= kBxStages && !mbar_wait(&bx_empty[b], ((it / kBxStages) - 1) & 1, p.status))) {
+          ok = false;
+          break;
+        }
+        const uint8_t *bp = tma_ring + s * kTmaStageBytes + kABytes;
+        uint8_t *bx = bx_ring + b * kBxBytes;
+        uint32_t w[(BN * BK / 16) / (32 * kExpWarps)];
+#pragma unroll
+        for (int i = 0; i < (BN * BK / 16) / (32 * kExpWarps); ++i) {
+          const int wi = et + 32 * kExpWarps * i;
+          w[i] = *reinterpret_cast<const uint32_t *>(bp + (wi >> 3) * 32 + (wi & 7) * 4);
+        }
+#pragma unroll
+        for (int i = 0; i < (BN * BK / 16) / (32 * kExpWarps); ++i) {
+          const int wi = et + 32 * kExpWarps * i;
+          const int r = wi >> 3, c = wi & 7;
+          *reinterpret_cast<uint4 *>(bx + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+              expand_word<PERM>(w[i]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bx_full[b]);
+      }
     }
   } else {
-    // ---- expansion: packed [256 rows x 32 B] -> int8 [256 x 128] K-major SW128
-    const int et = (warp - 2) * 32 + lane;
-    bool ok = true;
-    for (int kb = 0; kb < kblocks; ++kb) {
-      const int s = kb % kStages, it = kb / kStages;
-      if (!mbar_wait(&full_tma[s], it & 1, p.status)) {
-        ok = false;
-        break;
-      }
-      uint8_t *stage = smem + s * kStageBytes;
-      const uint8_t *bp = stage + kABytes + kBxBytes;
-      uint8_t *bx = stage + kABytes;
-#pragma unroll
-      for (int i = 0; i < (BN * BK / 16) / (32 * kExpWarps); ++i) {
-        const int wi = et + 32 * kExpWarps * i;
-        const int r = wi >> 3, c = wi & 7;
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(bp + r * 32 + c * 4);
-        const uint4 v = make_uint4(unpack_natural(w, 0), unpack_natural(w, 1),
-                                   unpack_natural(w, 2), unpack_natural(w, 3));
-        *reinterpret_cast<uint4 *>(bx + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full_x[s]);
-    }
-    // ---- epilogue: TMEM -> registers -> scale -> Y
-    if (ok && mbar_wait(done, 0, p.status)) {
+    // ---- epilogue warps 0-3: TMEM lane quadrant = warp
+    const int q = warp;
+    const float gamma = *p.gamma;
+    const bool vec_ok = (YK == kBF16) ? (p.N % 8 == 0) : (p.N % 4 == 0);
+    int tl = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tl) {
+      const int acc = tl & 1;
+      if (!mbar_wait(&acc_full[acc], (tl >> 1) & 1, p.status)) break;
       tc_fence_after();
-      const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-      const int half = (warp - 2) >> 2;       // which 128 columns
-      const int64_t m = m0 + q * 32 + lane;
-      const float r = (m < p.M) ? __fdiv_rn(*p.gamma, p.s[m]) : 0.0f;
-      const bool vec_ok = (YK == kBF16) ? (p.N % 8 == 0) : (p.N % 4 == 0);
+      const int64_t m = static_cast<int64_t>(tile / p.n_tiles) * BM + q * 32 + lane;
+      const int64_t n0 = static_cast<int64_t>(tile % p.n_tiles) * BN;
+      const float r = (m < p.M) ? __fdiv_rn(gamma, p.s[m]) : 0.0f;
+      const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * BN) +
+                             (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int cc = 0; cc < 8; ++cc) {
-        const int col = half * 128 + cc * 16;
+      for (int cc = 0; cc < BN / 16; ++cc) {
         uint32_t v[16];
-        tmem_ld16(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col), v);
+        tmem_ld16(t_row + static_cast<uint32_t>(cc * 16), v);
         tmem_wait_ld();
-        if (m < p.M && n0 + col < p.N) store16<YK, RELU2>(p, m, n0 + col, v, r, vec_ok);
+        if (m < p.M && n0 + cc * 16 < p.N) store16<YK, RELU2>(p, m, n0 + cc * 16, v, r, vec_ok);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem_d, kTmemCols);
+  if (warp == kWarpMma) tmem_dealloc(tmem_base, kTmemCols);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -246,27 +321,37 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YK, bool RELU2>
+template <int YK, bool RELU2, bool PERM>
 cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const PrefillParams &p,
                const LaunchCtx &ctx) {
-  auto kern = prefill_kernel<YK, RELU2>;
+  auto kern = prefill_kernel<YK, RELU2, PERM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(ceil_div(p.N, BN)), static_cast<unsigned>(ceil_div(p.M, BM)));
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const dim3 grid(static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms));
   return launch_k(kern, grid, dim3(kThreads), kSmemBytes, ctx, ta, tb, p);
+}
+
+template <bool PERM>
+cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const PrefillParams &p, int y_kind,
+                 bool relu2, const LaunchCtx &ctx) {
+  if (y_kind == kI32) return go<kI32, false, PERM>(ta, tb, p, ctx);
+  if (y_kind == kF32)
+    return relu2 ? go<kF32, true, PERM>(ta, tb, p, ctx) : go<kF32, false, PERM>(ta, tb, p, ctx);
+  return relu2 ? go<kBF16, true, PERM>(ta, tb, p, ctx) : go<kBF16, false, PERM>(ta, tb, p, ctx);
 }
 
 }  // namespace
 
 bool prefill_supported(int64_t M, int64_t N, int64_t K) {
-  return M >= 1 && N >= 1 && K % 64 == 0 && ceil_div(M, BM) < 65536 && ceil_div(N, BN) < (1LL << 31) &&
+  return M >= 1 && N >= 1 && K % 64 == 0 && ceil_div(M, BM) * ceil_div(N, BN) < (1LL << 31) &&
          encode_fn() != nullptr;
 }
 
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, bool /*weights_static*/, const LaunchCtx &ctx) {
+                           void *Y, int y_kind, bool xq_permuted, const LaunchCtx &ctx) {
   CUtensorMap ta, tb;
   if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                    static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -281,9 +366,10 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *pack
   p.M = M;
   p.N = N;
   p.K = K;
-  if (y_kind == kI32) return go<kI32, false>(ta, tb, p, ctx);
-  if (y_kind == kF32) return relu2 ? go<kF32, true>(ta, tb, p, ctx) : go<kF32, false>(ta, tb, p, ctx);
-  return relu2 ? go<kBF16, true>(ta, tb, p, ctx) : go<kBF16, false>(ta, tb, p, ctx);
+  p.m_tiles = static_cast<int>(ceil_div(M, BM));
+  p.n_tiles = static_cast<int>(ceil_div(N, BN));
+  return xq_permuted ? go_y<true>(ta, tb, p, y_kind, relu2, ctx)
+                     : go_y<false>(ta, tb, p, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet

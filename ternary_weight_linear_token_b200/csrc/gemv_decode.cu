@@ -10,10 +10,14 @@
 // they stream while the previous kernel in the stream finishes.  After the
 // wait the CTA quantises the activations per token (s = 127 / max|x|,
 // round half away, clamp +-127 -- identical to bitnet_quantize_act) into
-// shared memory, then 4 warps split K and run int8 mma.sync m16n8k32:
-// A = 16 weight rows x 32 k (unpacked from 2-bit codes in registers),
-// B = 32 k x 8 tokens.  Accumulation is exact int32; warps are reduced in
-// shared memory and the epilogue applies gamma / s and the optional ReLU^2.
+// shared memory: one token is spread over all 8 warps (each element loaded
+// once, amax reduced across the block), several tokens go one per warp.
+// Then the 8 warps split K into 64-element steps (balanced to within one
+// step) and run int8 mma.sync m16n8k32: A = 16 weight rows x 32 k (unpacked
+// from 2-bit codes in registers), B = 32 k x 8 tokens, two independent
+// accumulator chains per warp.  Accumulation is exact int32; the warps are
+// reduced in shared memory and the epilogue applies gamma / s and the
+// optional ReLU^2.
 //
 // Unpack: a 32-bit packed word holds element 16g + 4j + i at bits 8i + 2j.
 // Shifting the word by 0, 2, 16 or 18 and masking with 0x3333 puts four
@@ -22,7 +26,7 @@
 // weights for 3 instructions.  The four elements a shift selects are
 // {0,8,1,9}, {4,12,5,13}, {2,10,3,11}, {6,14,7,15}; the dot product does not
 // depend on the order of k, so the activations are stored in shared memory
-// in that same order (one 16-byte chunk per packed word).
+// in that same order (one 16-byte chunk per packed word, words in order).
 #include "common.cuh"
 #include "internal.h"
 
@@ -30,7 +34,7 @@ namespace bitnet {
 namespace {
 
 constexpr int kRows = 16;
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
@@ -49,19 +53,23 @@ struct DecodeParams {
   int weights_static;
 };
 
-// Smallest b >= bytes with b % 16 == 0 and b % 128 == 64: rows that far apart
-// put the 8 lanes of a 16-byte shared-memory access on distinct banks.
-__host__ __device__ constexpr int pad_row(int bytes) {
+// Smallest b >= bytes with b % 16 == 0 and b % 128 == r.
+__host__ __device__ constexpr int pad_to(int bytes, int r) {
   const int b = (bytes + 15) & ~15;
-  return b + (((64 - b % 128) % 128) + 128) % 128;
+  return b + (((r - b % 128) % 128) + 128) % 128;
 }
+// Weight rows 16 mod 128 bytes apart: the 8 rows x 4 consecutive words a warp
+// reads per step land on 32 distinct banks.  Token rows 64 mod 128 apart:
+// the two tokens x 4 chunks of a quarter-warp's 16-byte reads do too.
+int weight_row_bytes(int K) { return pad_to(K / 4, 16); }
+int token_row_bytes(int K) { return pad_to(K, 64); }
 
 __host__ __device__ constexpr int red_bytes(int mt) { return kWarps * mt * 32 * 16; }
 constexpr int kHeader = 256;  // mbarrier, per-token scales, amax partials
 
 size_t smem_bytes(int mt, int K) {
-  return kHeader + red_bytes(mt) + static_cast<size_t>(kRows) * pad_row(K / 4) +
-         static_cast<size_t>(8 * mt) * pad_row(K);
+  return kHeader + red_bytes(mt) + static_cast<size_t>(kRows) * weight_row_bytes(K) +
+         static_cast<size_t>(8 * mt) * token_row_bytes(K);
 }
 
 __device__ __forceinline__ uint32_t unpack_sel(uint32_t w, int shift) {
@@ -75,19 +83,6 @@ __device__ __forceinline__ void mma_16832(int (&c)[4], uint32_t a0, uint32_t a1,
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Shared-memory slot of packed word index W inside a token row: thread t of
-// a quad reads words 4t..4t+3 of a 16-word unit, one per step p; storing word
-// (16u + 4t + p) at slot (16u + 4p + t) makes each step's reads contiguous.
-__device__ __forceinline__ int x_slot(int W) {
-  const int u = W >> 4, r = W & 15;
-  return (u << 4) + ((r & 3) << 2) + (r >> 2);
-}
-
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
 }
 
 template <int KIND>
@@ -131,12 +126,95 @@ __device__ __forceinline__ void emit(const DecodeParams &p, int n, int m, int ac
   }
 }
 
+// One token quantised by the whole block: each 16-element chunk is loaded
+// once (up to kCache chunks per thread stay in registers for the second
+// use), the row's max |x| is reduced across the 8 warps.
+template <int XK>
+__device__ __forceinline__ float quantize_token_block(const DecodeParams &p, int m, uint8_t *xrow,
+                                                      float *amax_sh) {
+  constexpr int kCache = 2;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int words = p.K / 16;
+  const size_t base = static_cast<size_t>(m) * p.K;
+  float v[kCache][16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int c = 0; c < kCache; ++c) {
+    const int w = tid + c * kThreads;
+    if (w < words) {
+      load16<XK>(p.X, base + 16 * w, v[c]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
+    }
+  }
+  for (int w = tid + kCache * kThreads; w < words; w += kThreads) {
+    float t[16];
+    load16<XK>(p.X, base + 16 * w, t);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(t[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) amax_sh[warp] = amax;
+  __syncthreads();
+  amax = amax_sh[0];
+#pragma unroll
+  for (int i = 1; i < kWarps; ++i) amax = fmaxf(amax, amax_sh[i]);
+  const float sm = act_scale(amax);
+#pragma unroll
+  for (int c = 0; c < kCache; ++c) {
+    const int w = tid + c * kThreads;
+    if (w < words) {
+      int q[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[c][e], sm);
+      *reinterpret_cast<uint4 *>(xrow + 16 * w) = pack_permuted(q);
+    }
+  }
+  for (int w = tid + kCache * kThreads; w < words; w += kThreads) {
+    float t[16];
+    load16<XK>(p.X, base + 16 * w, t);
+    int q[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = quant_i8(t[e], sm);
+    *reinterpret_cast<uint4 *>(xrow + 16 * w) = pack_permuted(q);
+  }
+  return sm;
+}
+
+// One token quantised by one warp (used when the group has several tokens).
+template <int XK>
+__device__ __forceinline__ float quantize_token_warp(const DecodeParams &p, int m, uint8_t *xrow) {
+  const int lane = threadIdx.x & 31;
+  const int words = p.K / 16;
+  const size_t base = static_cast<size_t>(m) * p.K;
+  float amax = 0.0f;
+  for (int w = lane; w < words; w += 32) {
+    float t[16];
+    load16<XK>(p.X, base + 16 * w, t);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(t[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float sm = act_scale(amax);
+  for (int w = lane; w < words; w += 32) {
+    float t[16];
+    load16<XK>(p.X, base + 16 * w, t);
+    int q[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = quant_i8(t[e], sm);
+    *reinterpret_cast<uint4 *>(xrow + 16 * w) = pack_permuted(q);
+  }
+  return sm;
+}
+
 template <int MT, int XK, int YK, bool RELU2>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-  float *s_sh = reinterpret_cast<float *>(smem + 16);     // 32 per-token scales
-  float *amax_sh = reinterpret_cast<float *>(smem + 160); // kWarps partial maxima
+  float *s_sh = reinterpret_cast<float *>(smem + 16);      // 32 per-token scales
+  float *amax_sh = reinterpret_cast<float *>(smem + 160);  // kWarps partial maxima
   int4 *red = reinterpret_cast<int4 *>(smem + kHeader);
   uint8_t *wsh = smem + kHeader + red_bytes(MT);
   uint8_t *xsh = wsh + kRows * p.ws;
@@ -146,7 +224,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const int rows = min(kRows, p.N - n0);
   const uint32_t row_bytes = static_cast<uint32_t>(p.K) / 4;
   const int words = p.K / 16;
-  const int units = (words + 15) / 16;
+  const int steps = words / 4;  // 64-element steps (K % 64 == 0)
+  const int st0 = warp * steps / kWarps, st1 = (warp + 1) * steps / kWarps;
 
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -176,50 +255,26 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   for (int m0 = 0; m0 < p.M; m0 += p.tg) {
     const int mg = min(p.tg, p.M - m0);
     // ---- activations of this token group -> shared memory (permuted int8)
-    for (int t = 0; t < mg; ++t) {
-      const int m = m0 + t;
-      uint8_t *xrow = xsh + t * p.xs;
-      if (XK == kI8) {
-        const int8_t *src = static_cast<const int8_t *>(p.X) + static_cast<size_t>(m) * p.K;
-        for (int w = tid; w < words; w += kThreads) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * w);
-          uint4 o;
-          o.x = __byte_perm(v.x, v.z, 0x5140);
-          o.y = __byte_perm(v.y, v.w, 0x5140);
-          o.z = __byte_perm(v.x, v.z, 0x7362);
-          o.w = __byte_perm(v.y, v.w, 0x7362);
-          *reinterpret_cast<uint4 *>(xrow + 16 * x_slot(w)) = o;
-        }
-        if (tid == 0) s_sh[t] = p.s_in[m];
-      } else {
-        float amax = 0.0f;
-        for (int w = tid; w < words; w += kThreads) {
-          float v[16];
-          load16<XK>(p.X, static_cast<size_t>(m) * p.K + 16 * w, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        if (lane == 0) amax_sh[warp] = amax;
-        __syncthreads();
-        amax = fmaxf(fmaxf(amax_sh[0], amax_sh[1]), fmaxf(amax_sh[2], amax_sh[3]));
-        const float sm = act_scale(amax);
-        for (int w = tid; w < words; w += kThreads) {
-          float v[16];
-          load16<XK>(p.X, static_cast<size_t>(m) * p.K + 16 * w, v);
-          int q[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
-          uint4 o;
-          o.x = pack4(q[0], q[8], q[1], q[9]);
-          o.y = pack4(q[4], q[12], q[5], q[13]);
-          o.z = pack4(q[2], q[10], q[3], q[11]);
-          o.w = pack4(q[6], q[14], q[7], q[15]);
-          *reinterpret_cast<uint4 *>(xrow + 16 * x_slot(w)) = o;
-        }
-        if (tid == 0) s_sh[t] = sm;
-        __syncthreads();  // amax_sh is reused by the next token
+    if (XK == kI8) {
+      for (int i = tid; i < mg * words; i += kThreads) {
+        const int t = i / words, w = i - t * words;
+        const uint4 v = *reinterpret_cast<const uint4 *>(static_cast<const int8_t *>(p.X) +
+                                                         static_cast<size_t>(m0 + t) * p.K + 16 * w);
+        uint4 o;
+        o.x = __byte_perm(v.x, v.z, 0x5140);
+        o.y = __byte_perm(v.y, v.w, 0x5140);
+        o.z = __byte_perm(v.x, v.z, 0x7362);
+        o.w = __byte_perm(v.y, v.w, 0x7362);
+        *reinterpret_cast<uint4 *>(xsh + t * p.xs + 16 * w) = o;
+      }
+      if (tid < mg) s_sh[tid] = p.s_in[m0 + tid];
+    } else if (mg == 1) {
+      const float sm = quantize_token_block<XK>(p, m0, xsh, amax_sh);
+      if (tid == 0) s_sh[0] = sm;
+    } else {
+      for (int t = warp; t < mg; t += kWarps) {
+        const float sm = quantize_token_warp<XK>(p, m0 + t, xsh + t * p.xs);
+        if (lane == 0) s_sh[t] = sm;
       }
     }
     __syncthreads();
@@ -228,36 +283,37 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       waited = true;
     }
 
-    // ---- contraction: each warp takes 256-element units of K in turn
-    int c[MT][4];
+    // ---- contraction: warp w takes 64-element steps [st0, st1)
+    int c[MT][2][4];
 #pragma unroll
-    for (int tt = 0; tt < MT; ++tt) c[tt][0] = c[tt][1] = c[tt][2] = c[tt][3] = 0;
+    for (int tt = 0; tt < MT; ++tt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) c[tt][h][0] = c[tt][h][1] = c[tt][h][2] = c[tt][h][3] = 0;
     const int mt_active = (mg + 7) >> 3;
     if (weights_ok) {
-      for (int u = warp; u < units; u += kWarps) {
-        const int wbase = u * 16 + 4 * tq;
-        uint4 wa = make_uint4(0, 0, 0, 0), wb = make_uint4(0, 0, 0, 0);
-        if (wbase < words) {
-          wa = *reinterpret_cast<const uint4 *>(wsh + g * p.ws + 4 * wbase);
-          wb = *reinterpret_cast<const uint4 *>(wsh + (g + 8) * p.ws + 4 * wbase);
-        }
-        const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w};
-        const uint32_t wb_[4] = {wb.x, wb.y, wb.z, wb.w};
+      const uint32_t *wa_row = reinterpret_cast<const uint32_t *>(wsh + g * p.ws);
+      const uint32_t *wb_row = reinterpret_cast<const uint32_t *>(wsh + (g + 8) * p.ws);
+#pragma unroll 2
+      for (int st = st0; st < st1; ++st) {
+        const int word = 4 * st + tq;
+        const uint32_t wa = wa_row[word], wb = wb_row[word];
+        const uint32_t a0 = unpack_sel(wa, 0), a2 = unpack_sel(wa, 2);
+        const uint32_t a1 = unpack_sel(wb, 0), a3 = unpack_sel(wb, 2);
+        const uint32_t e0 = unpack_sel(wa, 16), e2 = unpack_sel(wa, 18);
+        const uint32_t e1 = unpack_sel(wb, 16), e3 = unpack_sel(wb, 18);
+        const int h = st & 1;
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          const uint32_t a0 = unpack_sel(wa_[pp], 0), a2 = unpack_sel(wa_[pp], 2);
-          const uint32_t a1 = unpack_sel(wb_[pp], 0), a3 = unpack_sel(wb_[pp], 2);
-          const uint32_t e0 = unpack_sel(wa_[pp], 16), e2 = unpack_sel(wa_[pp], 18);
-          const uint32_t e1 = unpack_sel(wb_[pp], 16), e3 = unpack_sel(wb_[pp], 18);
-#pragma unroll
-          for (int tt = 0; tt < MT; ++tt) {
-            if (tt < mt_active) {
-              uint4 b = make_uint4(0, 0, 0, 0);
-              if (tt * 8 + g < mg && wbase < words)
-                b = *reinterpret_cast<const uint4 *>(xsh + (tt * 8 + g) * p.xs +
-                                                     16 * (u * 16 + 4 * pp + tq));
-              mma_16832(c[tt], a0, a1, a2, a3, b.x, b.y);
-              mma_16832(c[tt], e0, e1, e2, e3, b.z, b.w);
+        for (int tt = 0; tt < MT; ++tt) {
+          if (tt < mt_active) {
+            uint4 b = make_uint4(0, 0, 0, 0);
+            if (tt * 8 + g < mg)
+              b = *reinterpret_cast<const uint4 *>(xsh + (tt * 8 + g) * p.xs + 16 * word);
+            if (h == 0) {
+              mma_16832(c[tt][0], a0, a1, a2, a3, b.x, b.y);
+              mma_16832(c[tt][0], e0, e1, e2, e3, b.z, b.w);
+            } else {
+              mma_16832(c[tt][1], a0, a1, a2, a3, b.x, b.y);
+              mma_16832(c[tt][1], e0, e1, e2, e3, b.z, b.w);
             }
           }
         }
@@ -265,10 +321,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     }
 #pragma unroll
     for (int tt = 0; tt < MT; ++tt)
-      red[(warp * MT + tt) * 32 + lane] = make_int4(c[tt][0], c[tt][1], c[tt][2], c[tt][3]);
+      red[(warp * MT + tt) * 32 + lane] =
+          make_int4(c[tt][0][0] + c[tt][1][0], c[tt][0][1] + c[tt][1][1],
+                    c[tt][0][2] + c[tt][1][2], c[tt][0][3] + c[tt][1][3]);
     __syncthreads();
 
-    // ---- reduce the 4 warps and apply the epilogue
+    // ---- reduce the 8 warps and apply the epilogue
     if (tid < 32 * mt_active) {
       const int tt = tid >> 5, l = tid & 31, gr = l >> 2, tc = l & 3;
       int4 sum = red[tt * 32 + l];
@@ -345,8 +403,8 @@ cudaError_t launch_decode(const void *X, int x_kind, const float *s, const uint8
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.ws = pad_row(static_cast<int>(K / 4));
-  p.xs = pad_row(static_cast<int>(K));
+  p.ws = weight_row_bytes(static_cast<int>(K));
+  p.xs = token_row_bytes(static_cast<int>(K));
   p.tg = 8 * mt;
   p.weights_static = weights_static ? 1 : 0;
   const size_t smem = smem_bytes(mt, static_cast<int>(K));

@@ -24,8 +24,10 @@ cudaError_t launch_quantize_weights(const void *W, int w_kind, int64_t N, int64_
                                     const LaunchCtx &ctx);
 
 // quant_act.cu
+// permuted: store each 16-element group of xq in the order the byte-permute
+// weight unpack produces (internal layout of the prefill kernel's A operand).
 cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
-                                float *s, const LaunchCtx &ctx);
+                                float *s, bool permuted, const LaunchCtx &ctx);
 cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
                             const LaunchCtx &ctx);
 
@@ -40,11 +42,12 @@ cudaError_t launch_generic(const int8_t *xq, const float *s, const uint8_t *pack
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                            void *Y, int y_kind, const LaunchCtx &ctx);
 
-// gemm_prefill.cu: tcgen05 tensor-core kernel, K % 64 == 0.
+// gemm_prefill.cu: tcgen05 tensor-core kernel, K % 64 == 0.  xq_permuted:
+// xq comes from launch_quantize_act(permuted = true).
 bool prefill_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, bool weights_static, const LaunchCtx &ctx);
+                           void *Y, int y_kind, bool xq_permuted, const LaunchCtx &ctx);
 
 // Launch helper: cudaLaunchKernelEx with the PDL attribute when ctx.pdl.
 template <typename... KArgs, typename... Args>

@@ -55,7 +55,7 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <int KIND>
+template <int KIND, bool PERM>
 __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const void *X, int64_t M,
                                                                          int64_t K, int8_t *xq,
                                                                          float *s) {
@@ -76,16 +76,13 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
     for (int64_t c = lane; c < chunks; c += 32) {
       float v[16];
       load16<KIND>(X, m * K + 16 * c, v);
-      uint32_t o[4];
+      int q[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          w |= (static_cast<uint32_t>(quant_i8(v[4 * q + b], sm)) & 0xFFu) << (8 * b);
-        o[q] = w;
-      }
-      *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
+      *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) =
+          PERM ? pack_permuted(q)
+               : make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                            pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
     }
     if (lane == 0) s[m] = sm;
   }
@@ -138,11 +135,14 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) rms_norm_kernel(const void *
 }  // namespace
 
 cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
-                                float *s, const LaunchCtx &ctx) {
+                                float *s, bool permuted, const LaunchCtx &ctx) {
   const dim3 grid(static_cast<unsigned>(ceil_div(M, kRowsPerCta)));
   const dim3 block(32 * kRowsPerCta);
-  if (x_kind == kF32) return launch_k(quantize_act_kernel<kF32>, grid, block, 0, ctx, X, M, K, xq, s);
-  return launch_k(quantize_act_kernel<kBF16>, grid, block, 0, ctx, X, M, K, xq, s);
+  if (x_kind == kF32)
+    return permuted ? launch_k(quantize_act_kernel<kF32, true>, grid, block, 0, ctx, X, M, K, xq, s)
+                    : launch_k(quantize_act_kernel<kF32, false>, grid, block, 0, ctx, X, M, K, xq, s);
+  return permuted ? launch_k(quantize_act_kernel<kBF16, true>, grid, block, 0, ctx, X, M, K, xq, s)
+                  : launch_k(quantize_act_kernel<kBF16, false>, grid, block, 0, ctx, X, M, K, xq, s);
 }
 
 cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,

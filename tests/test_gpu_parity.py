@@ -267,9 +267,14 @@ def test_prefill_workload_full_size_sampled(tw):
     got = bf16_bits_of(Y)[rows]
     assert_bf16_within_ulp(got, want)
     assert np.array_equal(got, want)
-    # the quantised activations the prefill path wrote into its workspace
-    xq_ws = np_of(ws[: 4096 * 2560]).view(np.int8).reshape(4096, 2560)
-    assert np.array_equal(xq_ws[rows], out["xq"])
+    # the quantised activations the prefill path wrote into its workspace, kept
+    # there in the K order of the kernel's weight unpack (inside each
+    # 16-element group: elements 0,8,1,9, 4,12,5,13, 2,10,3,11, 6,14,7,15)
+    perm = np.array([0, 8, 1, 9, 4, 12, 5, 13, 2, 10, 3, 11, 6, 14, 7, 15])
+    stored = np_of(ws[: 4096 * 2560]).view(np.int8).reshape(4096, 160, 16)
+    natural = np.empty_like(stored)
+    natural[:, :, perm] = stored
+    assert np.array_equal(natural.reshape(4096, 2560)[rows], out["xq"])
     # any-size property: a zero weight column block gives zero outputs
     assert tw.bitnet_get_device_status() == tw.OK
 
