@@ -3,8 +3,10 @@
 //
 // Every check runs before any CUDA call, so a rejected call has no side
 // effect and needs no GPU.  Paths of bitnet_w158a8_matmul:
+//   rows     M <= 4: one fused low-latency kernel (warp per output feature,
+//            dp4a; activation quantisation inside).
 //   decode   M <= 32, K % 64 == 0, the 16-row weight block fits in shared
-//            memory: one fused kernel (activation quantisation inside).
+//            memory: one fused kernel (int8 mma.sync; quantisation inside).
 //   prefill  otherwise, K % 64 == 0: bitnet_quantize_act into the workspace
 //            (unless xq is given), then the tcgen05 tensor-core kernel.
 //   generic  K % 64 != 0: quantise into the workspace, then the dp4a kernel.
@@ -89,7 +91,7 @@ bitnet_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : B
 // with float input).  Pure arithmetic: no CUDA call.
 size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
   if (M <= 0 || N <= 0 || K <= 0 || x_dtype == BITNET_I8) return 0;
-  if (decode_supported(M, N, K)) return 0;
+  if (rows_supported(M, N, K) || decode_supported(M, N, K)) return 0;
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
          align256(4 * static_cast<size_t>(M));
 }
@@ -195,6 +197,9 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
   const bool relu2 = epi == BITNET_EPI_RELU2;
   const bool wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
 
+  if (rows_supported(M, N, K))
+    return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                 wstatic, ctx));
   if (decode_supported(M, N, K))
     return from_cuda(launch_decode(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                    wstatic, ctx));

@@ -31,6 +31,12 @@ cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K,
 cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
                             const LaunchCtx &ctx);
 
+// gemv_rows.cu: lowest-latency kernel for 1 <= M <= 4 tokens, any K % 16 == 0.
+bool rows_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t *packed,
+                        const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2, void *Y,
+                        int y_kind, bool weights_static, const LaunchCtx &ctx);
+
 // gemv_decode.cu: fused decode kernel, M <= 32, K % 64 == 0.
 bool decode_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_decode(const void *X, int x_kind, const float *s, const uint8_t *packed,
