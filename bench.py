@@ -365,8 +365,8 @@ def main():
         return run_reference(args, world, rank)
 
     import torch
-    from ternary_weight_linear_token_b200 import build
-    build.build()
+    from __graft_entry__ import load_builder
+    load_builder().build()
     import ternary_weight_linear_token_b200 as tw
 
     dev = torch.device("cuda", local)

@@ -1,6 +1,10 @@
 """Build ``libbitnet158.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m ternary_weight_linear_token_b200.build [--force]
+    python ternary_weight_linear_token_b200/build.py [--force]
+
+Run it as a script or load it by file path (``load_builder`` in
+``__graft_entry__``): importing it through the package would first import the
+package, which loads the library it is meant to build.
 
 No fast-math: the quantisers and the epilogue rely on IEEE division,
 round-half-away ``roundf`` and uncontracted multiplies (``--fmad=false`` on

@@ -14,8 +14,8 @@ HEADER = os.path.join(ROOT, "include", "bitnet158.h")
 
 @pytest.fixture(scope="module")
 def tw():
-    from ternary_weight_linear_token_b200 import build
-    build.build()
+    from __graft_entry__ import load_builder
+    load_builder().build()
     import ternary_weight_linear_token_b200 as tw
     return tw
 

@@ -30,8 +30,8 @@ pytestmark = pytest.mark.gpu
 def tw():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    from ternary_weight_linear_token_b200 import build
-    build.build()
+    from __graft_entry__ import load_builder
+    load_builder().build()
     import ternary_weight_linear_token_b200 as tw
     return tw
 
