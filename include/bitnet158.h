@@ -156,6 +156,39 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                    uint32_t flags, bitnet_stream_t stream);
 
 /* ----------------------------------------------------------------------
+ * bitnet_w158a8_matmul for callers that cannot allocate device memory.
+ * (The pages on BitNet b1.58 have no counterpart of this entry point; it is
+ * a service of this library.)
+ *
+ * Some callers cannot give the library a workspace: a plugin inside a host
+ * framework that owns all device memory and hands out none, or a serving
+ * loop that must never call cudaMalloc because cudaMalloc can block until
+ * the whole device is idle.  This entry point takes the arguments of
+ * bitnet_w158a8_matmul without the workspace and uses a scratch array built
+ * into the library instead: BITNET_STATIC_SCRATCH_BYTES of device memory on
+ * every GPU that loads the library, held until the process exits.  It
+ * allocates nothing.
+ *   - A call whose scratch need, bitnet_w158a8_matmul_workspace_size(M, N,
+ *     K, x_dtype), is larger than BITNET_STATIC_SCRATCH_BYTES returns
+ *     BITNET_ERR_WORKSPACE and launches nothing.  The need is 0 for int8
+ *     input and for decode sizes, and about M*K bytes otherwise.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, which keeps whatever the
+ *     last call left in it; nothing in it needs to start at zero.  Calls
+ *     whose kernels overlap on the GPU (different streams or threads) race
+ *     on the array: keep them on one stream or otherwise serialised.
+ * ---------------------------------------------------------------------- */
+#define BITNET_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+bitnet_status bitnet_w158a8_matmul_noalloc(const void *X, bitnet_dtype x_dtype, const float *s,
+                                           const uint8_t *packed, const float *gamma, int64_t M,
+                                           int64_t N, int64_t K, bitnet_epilogue epi, void *Y,
+                                           bitnet_dtype y_dtype, uint32_t flags,
+                                           bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
  * Weightless per-token RMS normalisation, y = x / sqrt(mean_k(x^2) + 1e-6),
  * fp32 arithmetic, bf16 or fp32 in and out.  Glue between chained
  * BitLinears: the model card names "subln" normalisation (模型详情 -> 架构)

@@ -51,6 +51,8 @@ _SIGS = {
     "bitnet_w158a8_matmul": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST, _P, _SZ,
                               C.c_uint32, _P], _ST),
     "bitnet_rms_norm": ([_P, _ST, _I64, _I64, _P, _ST, _P], _ST),
+    "bitnet_w158a8_matmul_noalloc": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST,
+                                      C.c_uint32, _P], _ST),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -180,6 +182,38 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
                                   _DTYPE[Y.dtype], _ptr(workspace), ws_bytes,
                                   FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
     _check(st, "bitnet_w158a8_matmul")
+    return Y
+
+
+STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def bitnet_w158a8_matmul_noalloc(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                                 s: torch.Tensor | None = None, relu2: bool = False,
+                                 out_dtype: torch.dtype = torch.bfloat16,
+                                 Y: torch.Tensor | None = None, weights_static: bool = False,
+                                 stream=None) -> torch.Tensor:
+    """bitnet_w158a8_matmul with the library's built-in scratch array instead
+    of a workspace, for callers that cannot allocate device memory (the output
+    Y is still the caller's)."""
+    _dev(X, "X", (torch.float32, torch.bfloat16, torch.int8))
+    _dev(packed, "packed", (torch.uint8,))
+    _dev(gamma, "gamma", (torch.float32,))
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError(f"packed has {packed.shape[1]} bytes per row, expected K/4 = {K // 4}")
+    if s is not None:
+        _dev(s, "s", (torch.float32,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _dev(Y, "Y", (torch.float32, torch.bfloat16, torch.int32))
+    st = lib.bitnet_w158a8_matmul_noalloc(_ptr(X), _DTYPE[X.dtype], _ptr(s), _ptr(packed),
+                                          _ptr(gamma), M, N, K, EPI_RELU2 if relu2 else EPI_NONE,
+                                          _ptr(Y), _DTYPE[Y.dtype],
+                                          FLAG_WEIGHTS_STATIC if weights_static else 0,
+                                          _stream(stream))
+    _check(st, "bitnet_w158a8_matmul_noalloc")
     return Y
 
 
