@@ -8,16 +8,19 @@
 // features taken round-robin; K in 128-byte stages.
 //   warp 4      TMA producer: xq tile [128 x 128 B] (128-byte swizzle) and the
 //               packed weight tile [256 rows x 32 B] -- 2 bits per weight all
-//               the way from HBM into shared memory -- into a 6-stage ring.
-//   warps 6-13  expand each packed word into 16 int8 weights, stored as the
+//               the way from HBM into shared memory -- into a 5-stage ring.
+//   warps 6-21  expand each packed word into 16 int8 weights, stored as the
 //               K-major 128-byte-swizzled B operand in a 2-stage ring.
 //   warp 5      allocates 512 TMEM columns (two 256-column accumulators); one
 //               lane issues 4 MMAs (M=128, N=256, K=32) per stage and commits
 //               them to the barriers that free the TMA and B stages, and,
 //               after a tile's last stage, to the accumulator-full barrier.
 //   warps 0-3   epilogue: tcgen05.ld of the finished accumulator, y = acc *
-//               (gamma / s_m), optional ReLU^2, store; then release the
-//               accumulator, so tile i's epilogue overlaps tile i+1's MMAs.
+//               (gamma / s_m), optional ReLU^2; bf16 output goes through a
+//               128-byte-swizzled shared-memory staging block (32 rows x 64
+//               columns per warp, double-buffered) and a TMA tensor store,
+//               so HBM sees whole lines; then the accumulator is released,
+//               so tile i's epilogue overlaps tile i+1's MMAs.
 // Expansion: with activations quantised by this library (int8 in a K order
 // permuted inside each 16-element group) a packed word becomes 16 weights by
 // four byte-permute lookups (3 instructions per 4 weights); with int8
@@ -35,10 +38,10 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int kTmaStages = 6;
+constexpr int kTmaStages = 5;
 constexpr int kBxStages = 2;
 constexpr int kEpiWarps = 4;
-constexpr int kExpWarps = 8;
+constexpr int kExpWarps = 16;
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
 constexpr int kWarpExp0 = 6;
@@ -48,8 +51,11 @@ constexpr int kBpBytes = BN * BK / 4;
 constexpr int kTmaStageBytes = kABytes + kBpBytes;
 constexpr int kBxBytes = BN * BK;
 constexpr int kTmemCols = 2 * BN;
-constexpr size_t kSmemBytes =
-    1024 + static_cast<size_t>(kTmaStages) * kTmaStageBytes + kBxStages * kBxBytes + 256;
+constexpr int kStageRows = 32;                    // epilogue staging block: 32 rows
+constexpr int kStageCols = 64;                    // x 64 bf16 columns = 128-byte rows
+constexpr int kStageBytes = kStageRows * kStageCols * 2;
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kTmaStages) * kTmaStageBytes +
+                              kBxStages * kBxBytes + kEpiWarps * 2 * kStageBytes + 256;
 constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
 
 // Instruction descriptor: s8 x s8 -> s32, both operands K-major, M=128, N=256.
@@ -131,16 +137,18 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
                     unpack_natural(w, 3));
 }
 
-template <int YK, bool RELU2, bool PERM>
+template <int YK, bool RELU2, bool PERM, bool TMA_Y>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_y, const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *tma_ring = smem;
   uint8_t *bx_ring = smem + kTmaStages * kTmaStageBytes;
-  uint64_t *tma_full = reinterpret_cast<uint64_t *>(bx_ring + kBxStages * kBxBytes);
+  uint8_t *staging = bx_ring + kBxStages * kBxBytes;   // [kEpiWarps][2][32 x 128 B]
+  uint64_t *tma_full = reinterpret_cast<uint64_t *>(staging + kEpiWarps * 2 * kStageBytes);
   uint64_t *tma_empty = tma_full + kTmaStages;
   uint64_t *bx_full = tma_empty + kTmaStages;
   uint64_t *bx_empty = bx_full + kBxStages;
@@ -168,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    if (TMA_Y) prefetch_tmap(&tmap_y);
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_holder, kTmemCols);
@@ -267,27 +276,76 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp;
     const float gamma = *p.gamma;
     const bool vec_ok = (YK == kBF16) ? (p.N % 8 == 0) : (p.N % 4 == 0);
-    int tl = 0;
+    uint8_t *my_stage = staging + q * 2 * kStageBytes;
+    int tl = 0, stores = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tl) {
       const int acc = tl & 1;
       if (!mbar_wait(&acc_full[acc], (tl >> 1) & 1, p.status)) break;
       tc_fence_after();
-      const int64_t m = static_cast<int64_t>(tile / p.n_tiles) * BM + q * 32 + lane;
+      const int64_t m_base = static_cast<int64_t>(tile / p.n_tiles) * BM + q * 32;
+      const int64_t m = m_base + lane;
       const int64_t n0 = static_cast<int64_t>(tile % p.n_tiles) * BN;
       const float r = (m < p.M) ? __fdiv_rn(gamma, p.s[m]) : 0.0f;
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * BN) +
                              (static_cast<uint32_t>(q * 32) << 16);
+      if (TMA_Y) {
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 16; ++cc) {
-        uint32_t v[16];
-        tmem_ld16(t_row + static_cast<uint32_t>(cc * 16), v);
-        tmem_wait_ld();
-        if (m < p.M && n0 + cc * 16 < p.N) store16<YK, RELU2>(p, m, n0 + cc * 16, v, r, vec_ok);
+        for (int cb = 0; cb < BN / kStageCols; ++cb, ++stores) {
+          uint8_t *buf = my_stage + (stores & 1) * kStageBytes;
+          if (stores >= 2) {  // the store that last used this buffer has read it
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld16(t_row + static_cast<uint32_t>(cb * kStageCols + 32 * half),
+                      *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            tmem_ld16(t_row + static_cast<uint32_t>(cb * kStageCols + 32 * half + 16),
+                      *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+            tmem_wait_ld();
+            if (cb == BN / kStageCols - 1 && half == 1) {  // accumulator fully read
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {  // 8 columns = 16 bytes per chunk, swizzled
+              const int c = 4 * half + c4;
+              uint32_t h[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(
+                    epilogue_value(static_cast<int>(v[8 * c4 + 2 * e]), r, RELU2),
+                    epilogue_value(static_cast<int>(v[8 * c4 + 2 * e + 1]), r, RELU2));
+                h[e] = *reinterpret_cast<const uint32_t *>(&b);
+              }
+              *reinterpret_cast<uint4 *>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(h[0], h[1], h[2], h[3]);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, buf, static_cast<int32_t>(n0 + cb * kStageCols),
+                         static_cast<int32_t>(m_base));
+            bulk_commit();
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 16; ++cc) {
+          uint32_t v[16];
+          tmem_ld16(t_row + static_cast<uint32_t>(cc * 16), v);
+          tmem_wait_ld();
+          if (m < p.M && n0 + cc * 16 < p.N) store16<YK, RELU2>(p, m, n0 + cc * 16, v, r, vec_ok);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
     }
+    if (TMA_Y && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -309,37 +367,43 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                 CUtensorMapSwizzle swz) {
+                 CUtensorMapSwizzle swz,
+                 CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YK, bool RELU2, bool PERM>
-cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const PrefillParams &p,
-               const LaunchCtx &ctx) {
-  auto kern = prefill_kernel<YK, RELU2, PERM>;
+template <int YK, bool RELU2, bool PERM, bool TMA_Y>
+cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
+               const PrefillParams &p, const LaunchCtx &ctx) {
+  auto kern = prefill_kernel<YK, RELU2, PERM, TMA_Y>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   const dim3 grid(static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms));
-  return launch_k(kern, grid, dim3(kThreads), kSmemBytes, ctx, ta, tb, p);
+  return launch_k(kern, grid, dim3(kThreads), kSmemBytes, ctx, ta, tb, ty, p);
 }
 
 template <bool PERM>
-cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const PrefillParams &p, int y_kind,
-                 bool relu2, const LaunchCtx &ctx) {
-  if (y_kind == kI32) return go<kI32, false, PERM>(ta, tb, p, ctx);
+cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, bool tma_y,
+                 const PrefillParams &p, int y_kind, bool relu2, const LaunchCtx &ctx) {
+  if (y_kind == kI32) return go<kI32, false, PERM, false>(ta, tb, ty, p, ctx);
   if (y_kind == kF32)
-    return relu2 ? go<kF32, true, PERM>(ta, tb, p, ctx) : go<kF32, false, PERM>(ta, tb, p, ctx);
-  return relu2 ? go<kBF16, true, PERM>(ta, tb, p, ctx) : go<kBF16, false, PERM>(ta, tb, p, ctx);
+    return relu2 ? go<kF32, true, PERM, false>(ta, tb, ty, p, ctx)
+                 : go<kF32, false, PERM, false>(ta, tb, ty, p, ctx);
+  if (tma_y)
+    return relu2 ? go<kBF16, true, PERM, true>(ta, tb, ty, p, ctx)
+                 : go<kBF16, false, PERM, true>(ta, tb, ty, p, ctx);
+  return relu2 ? go<kBF16, true, PERM, false>(ta, tb, ty, p, ctx)
+               : go<kBF16, false, PERM, false>(ta, tb, ty, p, ctx);
 }
 
 }  // namespace
@@ -368,8 +432,15 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *pack
   p.K = K;
   p.m_tiles = static_cast<int>(ceil_div(M, BM));
   p.n_tiles = static_cast<int>(ceil_div(N, BN));
-  return xq_permuted ? go_y<true>(ta, tb, p, y_kind, relu2, ctx)
-                     : go_y<false>(ta, tb, p, y_kind, relu2, ctx);
+  // bf16 output with 16-byte rows goes out through TMA tensor stores
+  CUtensorMap ty;
+  const bool tma_y = y_kind == kBF16 && N % 8 == 0 &&
+                     make_map_2d(&ty, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                                 static_cast<uint64_t>(N) * 2, kStageCols, kStageRows,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  if (!tma_y) ty = ta;  // unused by the direct-store kernels
+  return xq_permuted ? go_y<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx)
+                     : go_y<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet
