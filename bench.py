@@ -253,14 +253,14 @@ def make_prefill(tw, torch, dev, l2_bytes):
     )
 
 
-def make_chain(tw, torch, dev, l2_bytes, layers=30):
+def make_chain(tw, torch, dev, l2_bytes, layers=30, persistent=False):
     import synth
     from ternary_weight_linear_token_b200.chain import DecodeChain
     ws = []
     for li in range(layers):
         ws.append([(torch.from_numpy(synth.layer_weights(li, p)).to(dev), synth.PROJECTIONS[p][3])
                    for p in range(4)])
-    chain = DecodeChain(ws, device=dev)
+    chain = DecodeChain(ws, device=dev, persistent=persistent)
     del ws
     x0 = synth.config_inputs("chain", weights=False)
     X = torch.from_numpy(x0["x_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
@@ -277,6 +277,8 @@ def make_chain(tw, torch, dev, l2_bytes, layers=30):
                             "o 2560->2560, up 2560->6912 + ReLU^2, down 6912->2560, rms norm",
                 "M": 1, "layers": layers, "x_dtype": "bf16", "y_dtype": "bf16",
                 "l2": f"inputs larger than L2: {wbytes / 1e6:.0f} MB of packed weights per token",
+                "mode": ("one persistent launch per token (bitnet_decode_chain)" if persistent
+                         else "one launch per projection and per normalisation"),
                 "timing": "CUDA graph of the timed steps"},
         kernel_key=None, kernel_files=[], e2e_inputs=lambda: (x0["x_bits"].view(np.int16), 5120, 5120),
     )
@@ -361,6 +363,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--chain-mode", choices=["persistent", "per-launch"], default="per-launch",
+                    help="chain workload: one persistent kernel per token, or one launch per step")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world, rank, local = dist_setup()
@@ -383,7 +387,8 @@ def main():
         pg = dist
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2**20))
-    w = MAKERS[args.workload](tw, torch, dev, l2)
+    extra = {"persistent": args.chain_mode == "persistent"} if args.workload == "chain" else {}
+    w = MAKERS[args.workload](tw, torch, dev, l2, **extra)
     stream = torch.cuda.Stream(dev)
 
     # warm-up (eager launches), then capture the timed steps in one graph

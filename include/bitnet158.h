@@ -200,6 +200,67 @@ bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, in
                               bitnet_dtype y_dtype, bitnet_stream_t stream);
 
 /* ----------------------------------------------------------------------
+ * A chain of M = 1 BitLinear projections in one launch.
+ *
+ * A decode step of BitNet b1.58 (the model card, 模型详情 -> 架构: a
+ * Transformer whose linear layers are all BitLinear, ReLU^2 in the FFN,
+ * a "subln" normalisation) runs its projections one after the other, each
+ * on the previous one's output re-quantised per token (the technical
+ * report's W1.58A8 BitLinear; 技术原理 of "Microsoft BitNet 深度研究报告").
+ * This call runs such a chain for one token in a single cooperative launch
+ * with one CTA per SM.  Every step computes exactly what
+ * bitnet_w158a8_matmul computes for M = 1 with bf16 input and bf16 output:
+ * same int8 activations and scale, same int32 accumulators, same epilogue.
+ *
+ * Step s reads the first K values of step s-1's output (of x0 for s = 0).
+ * With BITNET_STEP_NORM_IN it first applies the weightless RMS
+ * normalisation of bitnet_rms_norm to those K values, rounds them to bf16,
+ * and quantises that; X_normed (optional) receives them, so every link can
+ * be checked.  The normalisation's fp32 sum may be ordered differently from
+ * bitnet_rms_norm's (not part of the bit-exact contract).
+ *
+ *   steps      host array of n_steps descriptors (1 <= n_steps <=
+ *              BITNET_CHAIN_MAX_STEPS); read during the call only.
+ *   x0         bf16 [steps[0].K], device, 16-byte aligned.  Must not
+ *              overlap any output.
+ *   y_norm     bf16 [steps[n-1].N] or NULL: the RMS normalisation of the
+ *              last step's output (N % 16 == 0 and N <= 8192 when given).
+ *   workspace  >= bitnet_decode_chain_workspace_size(steps, n_steps) bytes,
+ *              16-byte aligned.  ZERO-FILLED before the first call; then
+ *              passed unchanged to every later call of a chain (the library
+ *              keeps a launch counter in it and tags its exchange words with
+ *              it).  After a call that reported BITNET_ERR_TIMEOUT, zero it
+ *              again.  Two chains must not run concurrently on one workspace.
+ * Per step: packed [N][K/4] and gamma as from bitnet_quantize_weights
+ * (packed 16-byte aligned); Y bf16 [N], 16-byte aligned; 1 <= N <= 2^22;
+ * K % 64 == 0, 64 <= K <= 8192 and K <= the previous step's N.  Shapes whose
+ * per-SM share of a step's packed rows does not fit twice in shared memory
+ * return BITNET_ERR_UNSUPPORTED_SHAPE.
+ * Every wait in the kernel is bounded; one that gives up records
+ * BITNET_ERR_TIMEOUT (read it with bitnet_get_device_status).
+ * ---------------------------------------------------------------------- */
+#define BITNET_CHAIN_MAX_STEPS 256
+#define BITNET_STEP_RELU2 1u   /* ReLU^2 epilogue */
+#define BITNET_STEP_NORM_IN 2u /* RMS-normalise the input before quantising it */
+
+typedef struct bitnet_chain_step {
+  const uint8_t *packed; /* [N][K/4] packed ternary codes, device */
+  const float *gamma;    /* device, 1 float */
+  int64_t N;             /* output features */
+  int64_t K;             /* input features */
+  uint32_t flags;        /* BITNET_STEP_RELU2 | BITNET_STEP_NORM_IN */
+  void *Y;               /* bf16 [N] output of this step, device */
+  void *X_normed;        /* bf16 [K] normalised input (NORM_IN steps only), or NULL */
+} bitnet_chain_step;
+
+/* 0 if the descriptors are invalid. */
+size_t bitnet_decode_chain_workspace_size(const bitnet_chain_step *steps, int n_steps);
+
+bitnet_status bitnet_decode_chain(const bitnet_chain_step *steps, int n_steps, const void *x0,
+                                  void *y_norm, void *workspace, size_t workspace_bytes,
+                                  bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
  * Status and diagnostics.
  * ---------------------------------------------------------------------- */
 /* Static English text for a status code (never NULL). */

@@ -54,6 +54,20 @@ _SIGS = {
     "bitnet_w158a8_matmul_noalloc": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST,
                                       C.c_uint32, _P], _ST),
 }
+
+
+class ChainStep(C.Structure):
+    """``bitnet_chain_step`` of the C header."""
+    _fields_ = [("packed", C.c_void_p), ("gamma", C.c_void_p), ("N", C.c_int64),
+                ("K", C.c_int64), ("flags", C.c_uint32), ("Y", C.c_void_p),
+                ("X_normed", C.c_void_p)]
+
+
+STEP_RELU2, STEP_NORM_IN = 1, 2
+CHAIN_MAX_STEPS = 256
+_SIGS["bitnet_decode_chain_workspace_size"] = ([C.POINTER(ChainStep), C.c_int], _SZ)
+_SIGS["bitnet_decode_chain"] = ([C.POINTER(ChainStep), C.c_int, _P, _P, _P, _SZ, _P], _ST)
+
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
     _f.argtypes = _args
@@ -230,3 +244,56 @@ def bitnet_rms_norm(X: torch.Tensor, Y: torch.Tensor | None = None,
                              _stream(stream))
     _check(st, "bitnet_rms_norm")
     return Y
+
+
+# ---------------------------------------------------------------- decode chain
+def bitnet_decode_chain_steps(steps) -> C.Array:
+    """Descriptor array for ``bitnet_decode_chain``: one dict per step with
+    ``packed`` [N, K/4] uint8, ``gamma`` [1] fp32, ``Y`` bf16 with N elements
+    and optionally ``relu2``, ``norm_in`` and ``X_normed`` (bf16, K elements).
+    The tensors must outlive every call that uses the array."""
+    arr = (ChainStep * len(steps))()
+    for i, d in enumerate(steps):
+        packed, gamma, Y = d["packed"], d["gamma"], d["Y"]
+        _dev(packed, f"steps[{i}].packed", (torch.uint8,))
+        _dev(gamma, f"steps[{i}].gamma", (torch.float32,))
+        _dev(Y, f"steps[{i}].Y", (torch.bfloat16,))
+        N, K = packed.shape[0], packed.shape[1] * 4
+        if Y.numel() != N:
+            raise ValueError(f"steps[{i}].Y has {Y.numel()} elements, expected N = {N}")
+        xn = d.get("X_normed")
+        if xn is not None:
+            _dev(xn, f"steps[{i}].X_normed", (torch.bfloat16,))
+            if xn.numel() != K:
+                raise ValueError(f"steps[{i}].X_normed has {xn.numel()} elements, expected K = {K}")
+        flags = (STEP_RELU2 if d.get("relu2") else 0) | (STEP_NORM_IN if d.get("norm_in") else 0)
+        arr[i] = ChainStep(packed.data_ptr(), gamma.data_ptr(), N, K, flags, Y.data_ptr(),
+                           None if xn is None else xn.data_ptr())
+    return arr
+
+
+def bitnet_decode_chain_workspace_size(steps) -> int:
+    arr = steps if isinstance(steps, C.Array) else bitnet_decode_chain_steps(steps)
+    return lib.bitnet_decode_chain_workspace_size(arr, len(arr))
+
+
+def bitnet_decode_chain(steps, x0: torch.Tensor, workspace: torch.Tensor,
+                        y_norm: torch.Tensor | None = None, stream=None) -> None:
+    """Runs a chain of M = 1 BitLinear projections in one launch.  ``steps``
+    is a list of step dicts (see ``bitnet_decode_chain_steps``) or a prebuilt
+    descriptor array; x0 is the bf16 input of the first step; ``workspace``
+    is a uint8 tensor of ``bitnet_decode_chain_workspace_size`` bytes,
+    zero-filled once and then kept for every call of this chain; y_norm
+    (optional, bf16) receives the RMS normalisation of the last output."""
+    arr = steps if isinstance(steps, C.Array) else bitnet_decode_chain_steps(steps)
+    _dev(x0, "x0", (torch.bfloat16,))
+    _dev(workspace, "workspace", (torch.uint8,))
+    if x0.numel() != arr[0].K:
+        raise ValueError(f"x0 has {x0.numel()} elements, expected K = {arr[0].K}")
+    if y_norm is not None:
+        _dev(y_norm, "y_norm", (torch.bfloat16,))
+        if y_norm.numel() != arr[len(arr) - 1].N:
+            raise ValueError("y_norm must have the last step's N elements")
+    st = lib.bitnet_decode_chain(arr, len(arr), _ptr(x0), _ptr(y_norm), _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+    _check(st, "bitnet_decode_chain")

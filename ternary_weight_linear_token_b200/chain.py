@@ -11,19 +11,27 @@ model card (BitNet b1.58 2B4T, 模型详情 -> 架构) names ReLU^2 in the FFN a
 normalisation between layers is the plain stand-in (without it the squared
 activations vanish within a few layers).
 
-Every step is a call of the C-ABI library on one stream; ``run`` launches
-5 kernels per layer and can be captured in a CUDA graph (``capture``).
+Two ways to run it, both through the C-ABI library on one stream and both
+capturable in a CUDA graph (``capture``):
+  * per launch (default): ``run`` makes one call per projection and one per
+    normalisation, 5 kernels per layer;
+  * persistent (``persistent=True``): ``run`` makes one call of
+    ``bitnet_decode_chain``, one kernel for the whole stack, with the
+    normalisation folded into the next layer's QKV projection.
+Both fill the same buffers (``outs``), so every link can be checked.
 """
 
 from __future__ import annotations
 
 import torch
 
-from . import bitnet_quantize_weights, bitnet_rms_norm, bitnet_w158a8_matmul
+from . import (bitnet_decode_chain, bitnet_decode_chain_steps, bitnet_decode_chain_workspace_size,
+               bitnet_quantize_weights, bitnet_rms_norm, bitnet_w158a8_matmul)
 
 
 class DecodeChain:
-    def __init__(self, weights, device="cuda:0", weights_static: bool = True):
+    def __init__(self, weights, device="cuda:0", weights_static: bool = True,
+                 persistent: bool = False):
         """weights: list over layers of a list of 4 (W [N, K] float tensor,
         relu2) pairs in the order qkv, o, up, down.  Weights are quantised on
         the device once, here."""
@@ -48,6 +56,19 @@ class DecodeChain:
             bufs.append(torch.empty((1, d), dtype=torch.bfloat16, device=self.device))  # norm out
             self.outs.append(bufs)
         self.graph = None
+        self.persistent = persistent
+        if persistent:
+            steps = []
+            for li, (proj, bufs) in enumerate(zip(self.layers, self.outs)):
+                for pi, p in enumerate(proj):
+                    step = dict(packed=p["packed"], gamma=p["gamma"], Y=bufs[pi], relu2=p["relu2"])
+                    if pi == 0 and li > 0:  # the previous layer's normalisation, folded in
+                        step.update(norm_in=True, X_normed=self.outs[li - 1][4])
+                    steps.append(step)
+            self._steps = bitnet_decode_chain_steps(steps)
+            self._keep = steps
+            self.workspace = torch.zeros(bitnet_decode_chain_workspace_size(self._steps),
+                                         dtype=torch.uint8, device=self.device)
 
     @property
     def packed_bytes(self) -> int:
@@ -60,6 +81,9 @@ class DecodeChain:
     def run(self, x0: torch.Tensor | None = None) -> torch.Tensor:
         if x0 is not None:
             self.x_in.copy_(x0)
+        if self.persistent:
+            bitnet_decode_chain(self._steps, self.x_in, self.workspace, y_norm=self.outs[-1][4])
+            return self.outs[-1][4]
         x = self.x_in
         for proj, bufs in zip(self.layers, self.outs):
             qkv, o, up, down = proj
@@ -86,4 +110,4 @@ class DecodeChain:
         return g
 
     def launches_per_token(self) -> int:
-        return 5 * len(self.layers)
+        return 1 if self.persistent else 5 * len(self.layers)

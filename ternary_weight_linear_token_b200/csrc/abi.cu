@@ -3,10 +3,10 @@
 //
 // Every check runs before any CUDA call, so a rejected call has no side
 // effect and needs no GPU.  Paths of bitnet_w158a8_matmul:
-//   rows     M <= 4: one fused low-latency kernel (warp per output feature,
+//   rows     M <= 8: one fused low-latency kernel (warp per output feature,
 //            dp4a; activation quantisation inside).
-//   decode   M <= 32, K % 64 == 0, the 16-row weight block fits in shared
-//            memory: one fused kernel (int8 mma.sync; quantisation inside).
+//   decode   9 <= M <= 32, K % 64 == 0: bitnet_quantize_act into the
+//            workspace (unless xq is given), then the int8 mma.sync kernel.
 //   prefill  otherwise, K % 64 == 0: bitnet_quantize_act into the workspace
 //            (unless xq is given), then the tcgen05 tensor-core kernel.
 //   generic  K % 64 != 0: quantise into the workspace, then the dp4a kernel.
@@ -87,13 +87,43 @@ bitnet_status check_k(int64_t K) {
 bitnet_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
 
 // Scratch the matmul needs: int8 xq [M][K] and fp32 s [M] whenever the
-// activation quantiser runs as its own kernel (prefill and generic paths
-// with float input).  Pure arithmetic: no CUDA call.
+// activation quantiser runs as its own kernel (decode, prefill and generic
+// paths with float input).  Pure arithmetic: no CUDA call.
 size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
   if (M <= 0 || N <= 0 || K <= 0 || x_dtype == BITNET_I8) return 0;
-  if (rows_supported(M, N, K) || decode_supported(M, N, K)) return 0;
+  if (rows_supported(M, N, K)) return 0;
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
          align256(4 * static_cast<size_t>(M));
+}
+
+static_assert(kStepRelu2 == BITNET_STEP_RELU2 && kStepNormIn == BITNET_STEP_NORM_IN,
+              "step flags");
+static_assert(kChainMaxSteps == BITNET_CHAIN_MAX_STEPS, "chain length");
+
+// Checks one chain descriptor list; BITNET_OK or the status to return.
+bitnet_status check_chain(const bitnet_chain_step *steps, int n_steps) {
+  if (steps == nullptr || n_steps < 1 || n_steps > BITNET_CHAIN_MAX_STEPS)
+    return BITNET_ERR_INVALID_ARG;
+  for (int s = 0; s < n_steps; ++s) {
+    const bitnet_chain_step &d = steps[s];
+    if (d.packed == nullptr || d.gamma == nullptr || d.Y == nullptr) return BITNET_ERR_INVALID_ARG;
+    if ((d.flags & ~(BITNET_STEP_RELU2 | BITNET_STEP_NORM_IN)) != 0) return BITNET_ERR_INVALID_ARG;
+    if (d.X_normed != nullptr && (d.flags & BITNET_STEP_NORM_IN) == 0) return BITNET_ERR_INVALID_ARG;
+    if (d.N < 1 || d.K < 1) return BITNET_ERR_INVALID_ARG;
+    if (d.N > (int64_t(1) << 22) || d.K % 64 != 0 || d.K < 64 || d.K > chain_max_k())
+      return BITNET_ERR_UNSUPPORTED_SHAPE;
+    if (s > 0 && d.K > steps[s - 1].N) return BITNET_ERR_INVALID_ARG;
+    if (!aligned(d.packed, 16) || !aligned(d.gamma, 4) || !aligned(d.Y, 16) ||
+        (d.X_normed != nullptr && !aligned(d.X_normed, 16)))
+      return BITNET_ERR_MISALIGNED;
+  }
+  return BITNET_OK;
+}
+
+size_t chain_workspace(const bitnet_chain_step *steps, int n_steps) {
+  size_t words = 0;
+  for (int s = 0; s < n_steps; ++s) words += static_cast<size_t>(chain_xch_words(steps[s].N));
+  return align256(kChainWorkspaceHeader + chain_stats_bytes(n_steps) + 8 * words);
 }
 
 }  // namespace
@@ -200,17 +230,13 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
   if (rows_supported(M, N, K))
     return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                  wstatic, ctx));
-  if (decode_supported(M, N, K))
-    return from_cuda(launch_decode(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                   wstatic, ctx));
-
-  (void)wstatic;  // the prefill and generic kernels read the weights after the wait
-  const bool prefill = prefill_supported(M, N, K);
+  const bool decode = decode_supported(M, N, K);
+  const bool prefill = !decode && prefill_supported(M, N, K);
   const int8_t *xq = static_cast<const int8_t *>(X);
   const float *sq = s;
   if (x_dtype != BITNET_I8) {
     // The prefill kernel takes its own quantiser's output in the K order of
-    // its fast weight unpack; the generic kernel wants natural order.
+    // its fast weight unpack; the decode and generic kernels want natural order.
     int8_t *wxq = static_cast<int8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                           align256(static_cast<size_t>(M) * K));
@@ -219,6 +245,9 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
     xq = wxq;
     sq = ws;
   }
+  if (decode)
+    return from_cuda(launch_decode(xq, BITNET_I8, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                   wstatic, ctx));
   if (prefill)
     return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                     x_dtype != BITNET_I8, ctx));
@@ -242,6 +271,44 @@ bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, in
   LaunchCtx ctx;
   if (bitnet_status st = device_ctx(stream, &ctx)) return st;
   return from_cuda(launch_rms_norm(X, x_dtype, M, K, Y, y_dtype, ctx));
+}
+
+size_t bitnet_decode_chain_workspace_size(const bitnet_chain_step *steps, int n_steps) {
+  if (check_chain(steps, n_steps) != BITNET_OK) return 0;
+  return chain_workspace(steps, n_steps);
+}
+
+bitnet_status bitnet_decode_chain(const bitnet_chain_step *steps, int n_steps, const void *x0,
+                                  void *y_norm, void *workspace, size_t workspace_bytes,
+                                  bitnet_stream_t stream) {
+  if (bitnet_status st = check_chain(steps, n_steps)) return st;
+  if (x0 == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x0, 16) || (y_norm != nullptr && !aligned(y_norm, 16))) return BITNET_ERR_MISALIGNED;
+  const int64_t n_last = steps[n_steps - 1].N;
+  if (y_norm != nullptr && (n_last % 16 != 0 || n_last > chain_max_k()))
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  // x0 is read by every CTA during the first step: no output may overlap it
+  const size_t x0_bytes = 2 * static_cast<size_t>(steps[0].K);
+  for (int s = 0; s < n_steps; ++s) {
+    if (overlap(x0, x0_bytes, steps[s].Y, 2 * static_cast<size_t>(steps[s].N)) ||
+        (steps[s].X_normed != nullptr &&
+         overlap(x0, x0_bytes, steps[s].X_normed, 2 * static_cast<size_t>(steps[s].K))))
+      return BITNET_ERR_INVALID_ARG;
+  }
+  if (y_norm != nullptr && overlap(x0, x0_bytes, y_norm, 2 * static_cast<size_t>(n_last)))
+    return BITNET_ERR_INVALID_ARG;
+  const size_t need = chain_workspace(steps, n_steps);
+  if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return BITNET_ERR_MISALIGNED;
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  ChainStep cs[kChainMaxSteps];
+  for (int s = 0; s < n_steps; ++s)
+    cs[s] = ChainStep{steps[s].packed, steps[s].gamma, steps[s].N, steps[s].K, steps[s].flags,
+                      steps[s].Y, steps[s].X_normed};
+  ChainPlan plan;
+  if (!chain_plan(cs, n_steps, ctx.num_sms, &plan)) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_chain(cs, n_steps, plan, x0, y_norm, n_last, workspace, ctx));
 }
 
 bitnet_status bitnet_get_device_status(bitnet_stream_t stream) {

@@ -373,18 +373,19 @@ cudaError_t dispatch_y(const DecodeParams &p, size_t smem, int y_kind, bool relu
                : launch_t<MT, XK, kBF16, false>(p, smem, ctx);
 }
 
+// The library quantises the activations of this path once, in their own
+// kernel, so the kernel is instantiated for int8 input only.
 template <int MT>
 cudaError_t dispatch_x(const DecodeParams &p, size_t smem, int x_kind, int y_kind, bool relu2,
                        const LaunchCtx &ctx) {
-  if (x_kind == kI8) return dispatch_y<MT, kI8>(p, smem, y_kind, relu2, ctx);
-  if (x_kind == kF32) return dispatch_y<MT, kF32>(p, smem, y_kind, relu2, ctx);
-  return dispatch_y<MT, kBF16>(p, smem, y_kind, relu2, ctx);
+  if (x_kind != kI8) return cudaErrorInvalidValue;
+  return dispatch_y<MT, kI8>(p, smem, y_kind, relu2, ctx);
 }
 
 }  // namespace
 
 bool decode_supported(int64_t M, int64_t N, int64_t K) {
-  return M >= 1 && M <= 32 && N >= 1 && K % 64 == 0 && N < (1LL << 31) &&
+  return M > 8 && M <= 32 && N >= 1 && K % 64 == 0 && N < (1LL << 31) &&
          smem_bytes(1, static_cast<int>(K)) <= static_cast<size_t>(kSmemLimit);
 }
 

@@ -1,20 +1,22 @@
-// gemv_rows.cu -- lowest-latency BitLinear forward for 1 to 4 tokens.
+// gemv_rows.cu -- lowest-latency BitLinear forward for 1 to 8 tokens.
 //
 // At this size the packed weights of a projection (1.6 to 4.4 MB for the
 // decode shapes) stream from HBM in well under a microsecond, so the time a
-// call takes is set by its serial latency.  This kernel keeps that chain
-// short: one warp per output feature n, 16 features per CTA.
+// call takes is set by its serial latency and by the busiest SM.  The grid
+// has one CTA per SM (up to 32 warps each, more CTAs only for very wide
+// projections), and each CTA owns a contiguous, balanced range of output
+// features (17 or 18 of N = 2560 on 148 SMs); warp w takes features w,
+// w + warps, ... of that range.
 //   1. Before waiting for the previous kernel in the stream (programmatic
 //      dependent launch), the CTA starts asynchronous copies (cp.async) of
-//      its 16 rows of packed weights into shared memory, when the caller
-//      flags the weights as static; otherwise right after the wait.
-//   2. After the wait, the CTA quantises the activations: every 16-element
-//      group is loaded once, the per-token max |x| is reduced with one
-//      redux.sync per warp and one shared-memory atomicMax (|x| >= 0, so its
-//      bit pattern orders like an unsigned integer), and the int8 values
-//      (s = 127 / amax, round half away, clamp +-127 -- identical to
-//      bitnet_quantize_act) go to shared memory in the K order of the
-//      unpack below.
+//      its rows of packed weights into shared memory, when the caller flags
+//      the weights as static; otherwise right after the wait.
+//   2. After the wait, the CTA quantises the activations, 8 elements per
+//      thread: each element is loaded once, the per-token max |x| is reduced
+//      with one redux.sync per warp and one block barrier, and the int8
+//      values (s = 127 / amax, round half away, clamp +-127 -- identical to
+//      bitnet_quantize_act) go to shared memory in the K order of the unpack
+//      below (neighbouring threads swap 4 bytes with one shuffle for that).
 //   3. Each lane takes words l, l+32, ... of its row (a 32-bit word holds
 //      element 16g + 4j + i at bits 8i + 2j; shifting by 0, 2, 16, 18 and
 //      masking with 0x3333 makes four byte-permute selectors that look the
@@ -26,15 +28,19 @@
 //      y = (float)acc * (gamma / s_t) and the optional ReLU^2 and stores y.
 // No tensor cores: with one token the contraction is 2 ops per weight byte
 // per token, far below what the SM's integer pipes sustain.
+//
+// Shared-memory K order of one 16-element group (16 bytes): the elements the
+// unpack pairs with selector shifts 0, 16, 2, 18 -- {0,8,1,9}, {2,10,3,11},
+// {4,12,5,13}, {6,14,7,15} -- so elements 0..7 of the group fill bytes 0..7
+// with the help of 4 bytes from elements 8..11, and vice versa.
 #include "common.cuh"
 #include "internal.h"
 
 namespace bitnet {
 namespace {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kMaxTok = 4;
+constexpr int kMaxWarps = 32;
+constexpr int kMaxTok = 8;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
 
@@ -45,17 +51,28 @@ struct RowsParams {
   const float *gamma;
   void *Y;
   int M, N, K;
-  int xs;  // shared-memory bytes per token row
-  int ws;  // shared-memory bytes per weight row
+  int ctas;      // grid size: CTA c owns rows [c*N/ctas, (c+1)*N/ctas)
+  int xs;        // shared-memory bytes per token row
+  int ws;        // shared-memory bytes per weight row
   int weights_static;
 };
 
-constexpr int kHeader = 128;  // kMaxTok scales, kMaxTok amax words
+// scales [kMaxTok], gamma/s [kMaxTok], then per-warp maxima [kMaxWarps][kMaxTok]
+constexpr int kHeader = 32 + 32 + kMaxWarps * kMaxTok * 4;
 int x_row_bytes(int K) { return (K + 127) / 128 * 128; }
 int w_row_bytes(int K) { return (K / 4 + 15) / 16 * 16; }
-size_t rows_smem(int M, int K) {
-  return kHeader + static_cast<size_t>(M) * x_row_bytes(K) +
-         static_cast<size_t>(kWarps) * w_row_bytes(K);
+// One CTA per SM, so that a wide projection never runs a second wave (two
+// such CTAs do not fit on one SM together), unless a CTA would own more than
+// kMaxRowsPerCta features; never more CTAs than features.
+constexpr int kMaxRowsPerCta = 64;
+int rows_ctas(int64_t N, int num_sms) {
+  const int64_t per_sm_rows = (N + num_sms - 1) / num_sms;
+  const int64_t ctas = num_sms * ((per_sm_rows + kMaxRowsPerCta - 1) / kMaxRowsPerCta);
+  return static_cast<int>(ctas < N ? ctas : N);
+}
+int rows_per_cta(int64_t N, int ctas) { return static_cast<int>((N + ctas - 1) / ctas); }
+size_t rows_smem(int M, int K, int rows) {
+  return kHeader + static_cast<size_t>(M) * x_row_bytes(K) + static_cast<size_t>(rows) * w_row_bytes(K);
 }
 
 __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
@@ -74,173 +91,221 @@ __device__ __forceinline__ void start_weight_copy(const RowsParams &p, int n0, i
   const int row_bytes = p.K / 4;
   if ((row_bytes & 15) == 0) {
     const int per_row = row_bytes / 16;
-    for (int i = threadIdx.x; i < rows * per_row; i += kThreads) {
+    for (int i = threadIdx.x; i < rows * per_row; i += blockDim.x) {
       const int r = i / per_row, c = i - r * per_row;
       cp_async16(wsh + r * p.ws + 16 * c, p.packed + static_cast<size_t>(n0 + r) * row_bytes + 16 * c);
     }
   } else {
     const int per_row = row_bytes / 4;
-    for (int i = threadIdx.x; i < rows * per_row; i += kThreads) {
+    for (int i = threadIdx.x; i < rows * per_row; i += blockDim.x) {
       const int r = i / per_row, c = i - r * per_row;
       cp_async4(wsh + r * p.ws + 4 * c, p.packed + static_cast<size_t>(n0 + r) * row_bytes + 4 * c);
     }
   }
 }
 
+// 8 consecutive activations (16- or 32-byte aligned) as fp32.
 template <int KIND>
-__device__ __forceinline__ void load16(const void *X, size_t idx, float (&v)[16]) {
+__device__ __forceinline__ void load8(const void *X, size_t idx, float (&v)[8]) {
   if (KIND == kF32) {
     const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(X) + idx);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 f = p[q];
-      v[4 * q] = f.x;
-      v[4 * q + 1] = f.y;
-      v[4 * q + 2] = f.z;
-      v[4 * q + 3] = f.w;
-    }
+    const float4 a = p[0], b = p[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   } else {
-    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(X) + idx);
+    const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(X) + idx);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint4 u = p[q];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        v[8 * q + 2 * h] = __uint_as_float(w[h] << 16);
-        v[8 * q + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
-      }
+    for (int h = 0; h < 4; ++h) {
+      v[2 * h] = __uint_as_float(w[h] << 16);
+      v[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
     }
   }
 }
 
-__device__ __forceinline__ int dot_word(uint32_t w, uint4 x, int acc) {
-  acc = __dp4a(static_cast<int>(__byte_perm(kTernaryLut, 0u, w & 0x3333u)), static_cast<int>(x.x), acc);
-  acc = __dp4a(static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 2) & 0x3333u)), static_cast<int>(x.y), acc);
-  acc = __dp4a(static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 16) & 0x3333u)), static_cast<int>(x.z), acc);
-  acc = __dp4a(static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 18) & 0x3333u)), static_cast<int>(x.w), acc);
+// Quantise one 8-element half-group and store it, with the partner lane's
+// help, in the unpack order.  Both lanes of a pair must call this together
+// (the shuffle needs the whole warp); `active` is false past the end of K.
+__device__ __forceinline__ void store_half_group(uint8_t *xrow, int chunk, const float (&v)[8],
+                                                 float sm, bool active) {
+  int q[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) q[e] = active ? quant_i8(v[e], sm) : 0;
+  const bool lo = (chunk & 1) == 0;  // elements 0..7 of the group (else 8..15)
+  const uint32_t a = pack4(q[0], q[1], q[2], q[3]);
+  const uint32_t b = pack4(q[4], q[5], q[6], q[7]);
+  // low half sends elements 4..7, high half sends elements 8..11
+  const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? b : a, 1);
+  if (!active) return;
+  uint2 o;
+  if (lo) {  // bytes 0..7: {0,8,1,9}, {2,10,3,11}
+    o.x = __byte_perm(a, other, 0x5140);
+    o.y = __byte_perm(a, other, 0x7362);
+  } else {   // bytes 8..15: {4,12,5,13}, {6,14,7,15}
+    o.x = __byte_perm(other, b, 0x5140);
+    o.y = __byte_perm(other, b, 0x7362);
+  }
+  *reinterpret_cast<uint2 *>(xrow + 8 * chunk) = o;
+}
+
+// The 16 int8 weights of a packed word, as four dp4a operands in the
+// shared-memory K order (selector shifts 0, 16, 2, 18).
+struct Unpacked {
+  int a, b, c, d;
+};
+__device__ __forceinline__ Unpacked unpack_word(uint32_t w) {
+  return {static_cast<int>(__byte_perm(kTernaryLut, 0u, w & 0x3333u)),
+          static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 16) & 0x3333u)),
+          static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 2) & 0x3333u)),
+          static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 18) & 0x3333u))};
+}
+__device__ __forceinline__ int dot_word(const Unpacked &q, uint4 x, int acc) {
+  acc = __dp4a(q.a, static_cast<int>(x.x), acc);
+  acc = __dp4a(q.b, static_cast<int>(x.y), acc);
+  acc = __dp4a(q.c, static_cast<int>(x.z), acc);
+  acc = __dp4a(q.d, static_cast<int>(x.w), acc);
   return acc;
 }
 
 template <int MT, int XK, int YK, bool RELU2>
-__global__ void __launch_bounds__(kThreads) rows_kernel(const RowsParams p) {
+__global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  float *s_sh = reinterpret_cast<float *>(smem);                   // kMaxTok scales
-  unsigned *amax_sh = reinterpret_cast<unsigned *>(smem + 16);     // kMaxTok |x| maxima (bits)
+  float *s_sh = reinterpret_cast<float *>(smem);                 // kMaxTok scales
+  float *r_sh = reinterpret_cast<float *>(smem + 32);            // kMaxTok gamma / s
+  float *wmax = reinterpret_cast<float *>(smem + 64);            // [kMaxWarps][kMaxTok]
   uint8_t *xsh = smem + kHeader;
-  uint8_t *wsh = xsh + MT * p.xs;
+  uint8_t *wsh = xsh + p.M * p.xs;  // the host sizes shared memory for p.M token rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * kWarps;
-  const int rows = min(kWarps, p.N - n0);
+  const int nwarps = blockDim.x >> 5;
+  const int n0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.N / p.ctas);
+  const int n1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.N / p.ctas);
+  const int rows = n1 - n0;
   const int words = p.K / 16;
 
-  if (tid < kMaxTok) amax_sh[tid] = 0u;
   if (p.weights_static) start_weight_copy(p, n0, rows, wsh);
-  __syncthreads();  // amax_sh zeroed before any atomicMax
   pdl_launch_dependents();
   pdl_wait();
   if (!p.weights_static) start_weight_copy(p, n0, rows, wsh);
 
   // ---- activations -> shared memory (int8, unpack order), per-token scales
   if (XK == kI8) {
-    for (int i = tid; i < MT * words; i += kThreads) {
+    for (int i = tid; i < p.M * words; i += blockDim.x) {
       const int t = i / words, w = i - t * words;
       const uint4 v = *reinterpret_cast<const uint4 *>(static_cast<const int8_t *>(p.X) +
                                                        static_cast<size_t>(t) * p.K + 16 * w);
       uint4 o;
       o.x = __byte_perm(v.x, v.z, 0x5140);
-      o.y = __byte_perm(v.y, v.w, 0x5140);
-      o.z = __byte_perm(v.x, v.z, 0x7362);
+      o.y = __byte_perm(v.x, v.z, 0x7362);
+      o.z = __byte_perm(v.y, v.w, 0x5140);
       o.w = __byte_perm(v.y, v.w, 0x7362);
       *reinterpret_cast<uint4 *>(xsh + t * p.xs + 16 * w) = o;
     }
-    if (tid < MT) s_sh[tid] = p.s_in[tid];
+    if (tid < p.M) {
+      s_sh[tid] = p.s_in[tid];
+      r_sh[tid] = __fdiv_rn(*p.gamma, p.s_in[tid]);
+    }
   } else {
-    float v0[MT][16];  // the thread's first group of each token, kept for the second use
-    unsigned amax[MT];
+    const int chunks = p.K / 8;
+    constexpr int kCached = MT <= 2 ? MT : 1;  // tokens whose first 8 elements stay in registers
+    float v0[kCached][8];
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
+      if (t >= p.M) break;
       float a = 0.0f;
-      if (tid < words) {
-        load16<XK>(p.X, static_cast<size_t>(t) * p.K + 16 * tid, v0[t]);
+      if (tid < chunks) {
+        float v[8];
+        load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(v0[t][e]));
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
+        if (t < kCached) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v0[t < kCached ? t : 0][e] = v[e];
+        }
       }
-      for (int w = tid + kThreads; w < words; w += kThreads) {
-        float v[16];
-        load16<XK>(p.X, static_cast<size_t>(t) * p.K + 16 * w, v);
+      for (int c = tid + blockDim.x; c < chunks; c += blockDim.x) {
+        float v[8];
+        load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * c, v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(v[e]));
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
       }
-      amax[t] = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int t = 0; t < MT; ++t) atomicMax(&amax_sh[t], amax[t]);
+      a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
+      if (lane == 0) wmax[warp * kMaxTok + t] = a;
     }
     __syncthreads();
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-      const float sm = act_scale(__uint_as_float(amax_sh[t]));
-      if (tid == 0) s_sh[t] = sm;
-      if (tid < words) {
-        int q[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) q[e] = quant_i8(v0[t][e], sm);
-        *reinterpret_cast<uint4 *>(xsh + t * p.xs + 16 * tid) = pack_permuted(q);
+      if (t >= p.M) break;
+      float a = 0.0f;
+      for (int i = 0; i < nwarps; ++i) a = fmaxf(a, wmax[i * kMaxTok + t]);
+      const float sm = act_scale(a);
+      if (tid == blockDim.x - 1) {  // a lane with no activation work in the common case
+        s_sh[t] = sm;
+        r_sh[t] = __fdiv_rn(*p.gamma, sm);
       }
-      for (int w = tid + kThreads; w < words; w += kThreads) {
-        float v[16];
-        load16<XK>(p.X, static_cast<size_t>(t) * p.K + 16 * w, v);
-        int q[16];
+      uint8_t *xrow = xsh + t * p.xs;
+      {
+        float v[8];
+        if (t < kCached) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
-        *reinterpret_cast<uint4 *>(xsh + t * p.xs + 16 * w) = pack_permuted(q);
+          for (int e = 0; e < 8; ++e) v[e] = v0[t < kCached ? t : 0][e];
+        } else if (tid < chunks) {
+          load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
+        }
+        store_half_group(xrow, tid, v, sm, tid < chunks);
+      }
+      for (int c0 = blockDim.x; c0 < chunks; c0 += blockDim.x) {  // whole warps iterate together
+        const int c = c0 + tid;
+        float v[8];
+        if (c < chunks) load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * c, v);
+        store_half_group(xrow, c, v, sm, c < chunks);
       }
     }
   }
   cp_async_commit_wait();
   __syncthreads();
-  if (warp >= rows) return;
 
-  // ---- dot products of row n0 + warp with each token
-  const uint32_t *wrow = reinterpret_cast<const uint32_t *>(wsh + warp * p.ws);
-  int acc[MT][2];
+  // ---- dot products: warp w takes rows w, w + nwarps, ... of the CTA's range
+  for (int rl = warp; rl < rows; rl += nwarps) {
+    const uint32_t *wrow = reinterpret_cast<const uint32_t *>(wsh + rl * p.ws);
+    int acc[MT][2];
 #pragma unroll
-  for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = 0;
-  int w = lane;
-  for (; w + 32 < words; w += 64) {
-    const uint32_t wa = wrow[w], wb = wrow[w + 32];
+    for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = 0;
+    int w = lane;
+    for (; w + 32 < words; w += 64) {
+      const Unpacked qa = unpack_word(wrow[w]), qb = unpack_word(wrow[w + 32]);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        if (t < p.M) {
+          acc[t][0] = dot_word(qa, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * w), acc[t][0]);
+          acc[t][1] = dot_word(qb, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * (w + 32)), acc[t][1]);
+        }
+      }
+    }
+    if (w < words) {
+      const Unpacked qa = unpack_word(wrow[w]);
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+        if (t < p.M)
+          acc[t][0] = dot_word(qa, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * w), acc[t][0]);
+    }
+    int res = 0;
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-      acc[t][0] = dot_word(wa, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * w), acc[t][0]);
-      acc[t][1] = dot_word(wb, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * (w + 32)), acc[t][1]);
+      const int a = __reduce_add_sync(0xffffffffu, acc[t][0] + acc[t][1]);
+      if (lane == t) res = a;
     }
-  }
-  if (w < words) {
-    const uint32_t wa = wrow[w];
-#pragma unroll
-    for (int t = 0; t < MT; ++t)
-      acc[t][0] = dot_word(wa, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * w), acc[t][0]);
-  }
-  int res = 0;
-#pragma unroll
-  for (int t = 0; t < MT; ++t) {
-    const int a = __reduce_add_sync(0xffffffffu, acc[t][0] + acc[t][1]);
-    if (lane == t) res = a;
-  }
-  if (lane < MT) {
-    const int n = n0 + warp;
-    const size_t o = static_cast<size_t>(lane) * p.N + n;
-    if (YK == kI32) {
-      static_cast<int *>(p.Y)[o] = res;
-    } else {
-      const float y = epilogue_value(res, __fdiv_rn(*p.gamma, s_sh[lane]), RELU2);
-      if (YK == kF32)
-        static_cast<float *>(p.Y)[o] = y;
-      else
-        static_cast<__nv_bfloat16 *>(p.Y)[o] = __float2bfloat16_rn(y);
+    if (lane < p.M) {
+      const size_t o = static_cast<size_t>(lane) * p.N + n0 + rl;
+      if (YK == kI32) {
+        static_cast<int *>(p.Y)[o] = res;
+      } else {
+        const float y = epilogue_value(res, r_sh[lane], RELU2);
+        if (YK == kF32)
+          static_cast<float *>(p.Y)[o] = y;
+        else
+          static_cast<__nv_bfloat16 *>(p.Y)[o] = __float2bfloat16_rn(y);
+      }
     }
   }
 }
@@ -253,8 +318,11 @@ cudaError_t launch_t(const RowsParams &p, size_t smem, const LaunchCtx &ctx) {
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  const dim3 grid(static_cast<unsigned>(ceil_div(p.N, kWarps)));
-  return launch_k(kern, grid, dim3(kThreads), smem, ctx, p);
+  const int rpc = rows_per_cta(p.N, p.ctas);
+  const int warps = rpc < kMaxWarps ? rpc : kMaxWarps;
+  // an even warp count keeps the activation half-group pairs in whole warps
+  return launch_k(kern, dim3(static_cast<unsigned>(p.ctas)), dim3(32 * (warps < 2 ? 2 : warps)),
+                  smem, ctx, p);
 }
 
 template <int MT, int XK>
@@ -277,8 +345,10 @@ cudaError_t dispatch_x(const RowsParams &p, size_t smem, int x_kind, int y_kind,
 }  // namespace
 
 bool rows_supported(int64_t M, int64_t N, int64_t K) {
-  return M >= 1 && M <= kMaxTok && N >= 1 && N < (1LL << 31) && K % 16 == 0 &&
-         rows_smem(static_cast<int>(M), static_cast<int>(K)) <= static_cast<size_t>(kSmemLimit);
+  if (M < 1 || M > kMaxTok || N < 1 || N >= (1LL << 31) || K % 16 != 0 || K > (1 << 20)) return false;
+  // worst case rows per CTA on a device with at least 16 SMs
+  const int rpc = rows_per_cta(N, rows_ctas(N, 16));
+  return rows_smem(static_cast<int>(M), static_cast<int>(K), rpc) <= static_cast<size_t>(kSmemLimit);
 }
 
 cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t *packed,
@@ -293,16 +363,16 @@ cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
+  p.ctas = rows_ctas(N, ctx.num_sms);
   p.xs = x_row_bytes(static_cast<int>(K));
   p.ws = w_row_bytes(static_cast<int>(K));
   p.weights_static = weights_static ? 1 : 0;
-  const size_t smem = rows_smem(static_cast<int>(M), static_cast<int>(K));
-  switch (M) {
-    case 1: return dispatch_x<1>(p, smem, x_kind, y_kind, relu2, ctx);
-    case 2: return dispatch_x<2>(p, smem, x_kind, y_kind, relu2, ctx);
-    case 3: return dispatch_x<3>(p, smem, x_kind, y_kind, relu2, ctx);
-    default: return dispatch_x<4>(p, smem, x_kind, y_kind, relu2, ctx);
-  }
+  const size_t smem = rows_smem(static_cast<int>(M), static_cast<int>(K), rows_per_cta(N, p.ctas));
+  if (smem > static_cast<size_t>(kSmemLimit)) return cudaErrorInvalidValue;
+  if (M == 1) return dispatch_x<1>(p, smem, x_kind, y_kind, relu2, ctx);
+  if (M == 2) return dispatch_x<2>(p, smem, x_kind, y_kind, relu2, ctx);
+  if (M <= 4) return dispatch_x<4>(p, smem, x_kind, y_kind, relu2, ctx);
+  return dispatch_x<8>(p, smem, x_kind, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet

@@ -55,6 +55,36 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *pack
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                            void *Y, int y_kind, bool xq_permuted, const LaunchCtx &ctx);
 
+// chain.cu: persistent M = 1 chain of BitLinear projections (one
+// cooperative launch).  Step flags mirror BITNET_STEP_*.
+constexpr int kChainMaxSteps = 256;
+constexpr int kStepRelu2 = 1;
+constexpr int kStepNormIn = 2;
+constexpr size_t kChainWorkspaceHeader = 256;  // launch counter, finished-CTA counter
+constexpr int kChainMaxCtas = 256;              // CTAs of one chain launch, at most
+// Per-step, per-CTA records (two tagged 64-bit words: max |y|, sum y^2),
+// after the header; they double as the CTA's "outputs are out" flag.
+inline size_t chain_stats_bytes(int n_steps) { return static_cast<size_t>(n_steps) * kChainMaxCtas * 16; }
+struct ChainStep {
+  const uint8_t *packed;
+  const float *gamma;
+  int64_t N, K;
+  uint32_t flags;
+  void *Y;
+  void *Xn;
+};
+struct ChainPlan {
+  int ctas, slots, slot_bytes, xq_bytes, ystage_bytes;
+  size_t smem;
+};
+// 64-bit exchange words of one step's output: two bf16 values each.
+inline int64_t chain_xch_words(int64_t N) { return (N + 1) / 2; }
+int chain_max_k();
+bool chain_plan(const ChainStep *steps, int n_steps, int num_sms, ChainPlan *plan);
+cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &plan,
+                         const void *x0, void *y_norm, int64_t y_norm_n, void *workspace,
+                         const LaunchCtx &ctx);
+
 // Launch helper: cudaLaunchKernelEx with the PDL attribute when ctx.pdl.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,

@@ -94,11 +94,13 @@ def test_matmul_rejects_bad_arguments(tw):
 
 def test_workspace_sizes(tw):
     f = tw.lib.bitnet_w158a8_matmul_workspace_size
-    assert f(1, 2560, 2560, tw.BF16) == 0          # decode: fused, no scratch
-    assert f(32, 2560, 6912, tw.BF16) == 0
+    assert f(1, 2560, 2560, tw.BF16) == 0          # decode, M <= 8: fused, no scratch
+    assert f(8, 6912, 2560, tw.F32) == 0
+    assert f(32, 2560, 6912, tw.BF16) == 32 * 6912 + 256   # M > 8: quantised once
     assert f(4096, 6912, 2560, tw.I8) == 0          # xq given
     assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4
-    assert f(5, 64, 48, tw.F32) == 256 + 256        # generic path (K % 64 != 0)
+    assert f(5, 64, 48, tw.F32) == 0                # M <= 8: fused low-latency kernel, any K
+    assert f(9, 64, 48, tw.F32) == 512 + 256        # generic path (M > 8, K % 64 != 0)
     assert tw.lib.bitnet_quantize_weights_workspace_size(2560, 2560) == 2560 * 8
     assert tw.lib.bitnet_quantize_weights_workspace_size(3, 16) == 256
 
@@ -121,3 +123,54 @@ def test_quantizers_reject_bad_arguments(tw):
     assert r(A, 1, 4, 64, A, 0, None) == tw.ERR_INVALID_ARG             # in place, dtype change
     assert r(A, 1, 4, 64, C.c_void_p(0x10000010), 1, None) == tw.ERR_INVALID_ARG
     assert r(A, 1, 0, 64, B, 1, None) == tw.OK
+
+
+def chain(tw, shapes, flags=None, xn=None):
+    """Descriptor array with fake aligned device addresses."""
+    arr = (tw.ChainStep * len(shapes))()
+    for i, (N, K) in enumerate(shapes):
+        f = 0 if flags is None else flags[i]
+        x = None if xn is None else xn[i]
+        arr[i] = tw.ChainStep(0x20000000 + (i << 20), 0x40000000 + 256 * i, N, K, f,
+                              0x60000000 + (i << 20), x)
+    return arr
+
+
+def dc(tw, arr, n=None, x0=A, y=None, ws=WS, wsb=1 << 20):
+    return tw.lib.bitnet_decode_chain(arr, len(arr) if n is None else n, x0, y, ws, wsb, None)
+
+
+def test_decode_chain_rejects_bad_arguments(tw):
+    ok = chain(tw, [(3840, 2560), (2560, 2560), (6912, 2560), (2560, 6912)])
+    assert dc(tw, ok, n=0) == tw.ERR_INVALID_ARG
+    assert dc(tw, ok, n=257) == tw.ERR_INVALID_ARG
+    assert dc(tw, ok, x0=None) == tw.ERR_INVALID_ARG
+    assert dc(tw, ok, x0=MIS) == tw.ERR_MISALIGNED
+    assert dc(tw, chain(tw, [(64, 96)])) == tw.ERR_UNSUPPORTED_SHAPE       # K % 64
+    assert dc(tw, chain(tw, [(64, 8256)])) == tw.ERR_UNSUPPORTED_SHAPE     # K > 8192
+    assert dc(tw, chain(tw, [(100, 64), (64, 128)])) == tw.ERR_INVALID_ARG  # K > previous N
+    assert dc(tw, chain(tw, [(0, 64)])) == tw.ERR_INVALID_ARG
+    assert dc(tw, chain(tw, [(64, 64)], flags=[4])) == tw.ERR_INVALID_ARG
+    # X_normed without the normalisation flag
+    assert dc(tw, chain(tw, [(64, 64)], xn=[0x70000000])) == tw.ERR_INVALID_ARG
+    assert dc(tw, chain(tw, [(64, 64)], flags=[2], xn=[0x70000008])) == tw.ERR_MISALIGNED
+    # y_norm needs N % 16 == 0
+    assert dc(tw, chain(tw, [(100, 64)]), y=C.c_void_p(0x70000000)) == tw.ERR_UNSUPPORTED_SHAPE
+    # an output overlapping the chain input
+    assert dc(tw, chain(tw, [(64, 64)]), x0=C.c_void_p(0x60000000)) == tw.ERR_INVALID_ARG
+    need = tw.lib.bitnet_decode_chain_workspace_size(ok, 4)
+    assert dc(tw, ok, wsb=need - 1) == tw.ERR_WORKSPACE
+    assert dc(tw, ok, ws=None) == tw.ERR_WORKSPACE
+    assert dc(tw, ok, ws=C.c_void_p(0x50000008), wsb=need) == tw.ERR_MISALIGNED
+
+
+def test_decode_chain_workspace_size(tw):
+    f = tw.lib.bitnet_decode_chain_workspace_size
+    layer = [(3840, 2560), (2560, 2560), (6912, 2560), (2560, 6912)]
+    # 256-byte header, one 16-byte record per CTA (up to 256) per step, then
+    # one 8-byte word per two outputs of every step
+    words = sum((n + 1) // 2 for n, _ in layer)
+    assert f(chain(tw, layer), 4) == (256 + 4 * 4096 + 8 * words + 255) // 256 * 256
+    assert f(chain(tw, [(333, 64)]), 1) == 5888      # 256 + 4096 + 8 * 167 = 5688, rounded up
+    assert f(chain(tw, [(64, 40)]), 1) == 0          # invalid descriptors
+    assert f(chain(tw, layer * 30), 120) > 0

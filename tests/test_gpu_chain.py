@@ -1,0 +1,156 @@
+"""The persistent decode chain (bitnet_decode_chain) against the CPU oracle,
+link by link: every step's bf16 output must equal the oracle's BitLinear of
+the step's actual bf16 input (bit-exact); a normalised input (BITNET_STEP_NORM_IN)
+must be within 1 bf16 ulp of the oracle's RMS normalisation of the previous
+output, and the oracle's BitLinear is then fed the kernel's own normalised
+values.  Shapes cover odd N (a half-filled last exchange word), K smaller than
+the previous N, CTAs that own no row of a step (N < number of SMs), both
+epilogues, repeated launches on one workspace and CUDA-graph replay."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import DEV, assert_bf16_within_ulp, bf16_bits_of, bf16_t, f32_t, np_of
+from oracle import ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tw():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from __graft_entry__ import load_builder
+    load_builder().build()
+    import ternary_weight_linear_token_b200 as tw
+    return tw
+
+
+def build_chain(tw, specs, seed):
+    """specs: (N, K, relu2, norm_in) per step -> step dicts and latent weights."""
+    rng = np.random.default_rng(seed)
+    steps, Ws = [], []
+    for N, K, relu2, norm in specs:
+        W = synth.latent_weights(rng, N, K)
+        packed, gamma = tw.bitnet_quantize_weights(f32_t(W))
+        st = dict(packed=packed, gamma=gamma, relu2=relu2,
+                  Y=torch.full((N,), float("nan"), dtype=torch.bfloat16, device=DEV))
+        if norm:
+            st.update(norm_in=True, X_normed=torch.empty(K, dtype=torch.bfloat16, device=DEV))
+        steps.append(st)
+        Ws.append(W)
+    return steps, Ws
+
+
+def x0_bits(K, seed):
+    x = np.random.default_rng(seed).standard_t(3, K).astype(np.float32)
+    return synth.f32_to_bf16_bits(x)
+
+
+def check_links(steps, Ws, x0, y_norm=None):
+    prev = x0
+    for i, (st, W) in enumerate(zip(steps, Ws)):
+        N, K = st["packed"].shape[0], st["packed"].shape[1] * 4
+        po, go = ref.quantize_weights(W)
+        assert np.array_equal(np_of(st["packed"]), po), i
+        xin = prev[:K]
+        if st.get("norm_in"):
+            xn = bf16_bits_of(st["X_normed"])
+            want_n = ref.to_bf16(ref.rms_norm(synth.bf16_bits_to_f32(xin)[None, :]))[0]
+            assert_bf16_within_ulp(xn, want_n, 1)
+            xin = xn
+        want = ref.to_bf16(ref.bitlinear(synth.bf16_bits_to_f32(xin)[None, :], po, go, N,
+                                         relu2=st["relu2"])["y"])[0]
+        got = bf16_bits_of(st["Y"])
+        bad = np.flatnonzero(got != want)
+        assert bad.size == 0, (f"step {i}: {bad.size} of {N} outputs differ, first at {bad[:4]}: "
+                               f"got {got[bad[:4]]} want {want[bad[:4]]}")
+        prev = got
+    if y_norm is not None:
+        want = ref.to_bf16(ref.rms_norm(synth.bf16_bits_to_f32(prev)[None, :]))[0]
+        assert_bf16_within_ulp(bf16_bits_of(y_norm), want, 1)
+    return prev
+
+
+# (N, K, relu2, norm_in)
+SHAPES_A = [(333, 256, True, False),     # odd N: the last exchange word holds one value
+            (1000, 320, False, True),    # K < previous N; normalised input
+            (5000, 960, True, False),    # wide: ~34 rows per CTA
+            (64, 4992, False, True),     # fewer rows than CTAs
+            (8192, 64, True, False),     # the largest K the next step may use
+            (160, 8192, False, True)]    # K = 8192
+SHAPES_B = [(3840, 2560, False, False), (2560, 2560, False, False), (6912, 2560, True, False),
+            (2560, 6912, False, False), (1, 2560, False, True)]  # one output row
+
+
+@pytest.mark.parametrize("specs,seed,final_norm", [(SHAPES_A, 11, True), (SHAPES_B, 12, False)],
+                         ids=["ragged", "one_layer_then_one_row"])
+def test_decode_chain_links(tw, specs, seed, final_norm):
+    steps, Ws = build_chain(tw, specs, seed)
+    arr = tw.bitnet_decode_chain_steps(steps)
+    ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
+    y_norm = (torch.empty(specs[-1][0], dtype=torch.bfloat16, device=DEV) if final_norm else None)
+    for launch in range(3):  # the launch counter in the workspace advances every time
+        x0 = x0_bits(specs[0][1], seed + launch)
+        for st in steps:
+            st["Y"].fill_(float("nan"))
+        tw.bitnet_decode_chain(arr, bf16_t(x0), ws, y_norm=y_norm)
+        torch.cuda.synchronize()
+        check_links(steps, Ws, x0, y_norm)
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
+def test_decode_chain_graph_replay(tw):
+    """Captured in a CUDA graph, each replay is a new launch (new tag) and
+    recomputes every link from the current input."""
+    steps, Ws = build_chain(tw, SHAPES_A[:3], 21)
+    arr = tw.bitnet_decode_chain_steps(steps)
+    ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
+    x_in = torch.empty(SHAPES_A[0][1], dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        x_in.copy_(bf16_t(x0_bits(SHAPES_A[0][1], 0)))
+        tw.bitnet_decode_chain(arr, x_in, ws)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        tw.bitnet_decode_chain(arr, x_in, ws)
+    for r in range(3):
+        x0 = x0_bits(SHAPES_A[0][1], 100 + r)
+        x_in.copy_(bf16_t(x0))
+        g.replay()
+        torch.cuda.synchronize()
+        check_links(steps, Ws, x0)
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
+def test_decode_chain_matches_per_launch_chain(tw):
+    """Two layers of the 30-layer stack run both ways: the BitLinear links
+    agree with the oracle in both, and where the normalisations agree bit for
+    bit, so do all later outputs."""
+    from ternary_weight_linear_token_b200.chain import DecodeChain
+    layers = [[(f32_t(synth.layer_weights(li, p)), synth.PROJECTIONS[p][3]) for p in range(4)]
+              for li in range(2)]
+    x0 = synth.config_inputs("chain", weights=False)
+    x = bf16_t(x0["x_bits"])
+    per = DecodeChain(layers)
+    per.run(x)
+    pers = DecodeChain(layers, persistent=True)
+    pers.run(x)
+    torch.cuda.synchronize()
+    # the first layer has no normalisation: identical outputs
+    for pi in range(4):
+        assert np.array_equal(bf16_bits_of(per.outs[0][pi]), bf16_bits_of(pers.outs[0][pi])), pi
+    # every persistent link against the oracle
+    steps = [dict(packed=p["packed"], relu2=p["relu2"], Y=pers.outs[li][pi].view(-1))
+             for li, proj in enumerate(pers.layers) for pi, p in enumerate(proj)]
+    for li in range(1, 2):
+        steps[4 * li].update(norm_in=True, X_normed=pers.outs[li - 1][4].view(-1))
+    Ws = [synth.layer_weights(li, p) for li in range(2) for p in range(4)]
+    check_links(steps, Ws, x0["x_bits"].reshape(-1), pers.outs[-1][4].view(-1))
+    assert tw.bitnet_get_device_status() == tw.OK

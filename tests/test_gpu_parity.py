@@ -104,13 +104,13 @@ def test_quantize_act_bitexact(tw, name, x, dtype):
 
 
 # --------------------------------------------------------------- matmul
-# (M, N, K): low-latency shapes (M <= 4, any K % 16 == 0), decode shapes
-# (M <= 32, K % 64 == 0), prefill shapes on one CTA (M <= 128) and on CTA
-# pairs (M > 128, including a half-empty last pair and ragged M, N, K),
-# generic shapes (M > 4, K % 64 != 0).
+# (M, N, K): low-latency shapes (M <= 8, any K % 16 == 0, several CTAs per
+# SM, K beyond the register window), decode shapes (8 < M <= 32, K % 64 ==
+# 0), prefill shapes (several 128 x 256 tiles, ragged M, N, K), generic
+# shapes (M > 8, K % 64 != 0).
 SHAPES = [
     (1, 272, 320), (2, 275, 320), (3, 17, 64), (4, 40, 48), (1, 33, 8704), (4, 21, 10240),
-    (2, 5, 16), (5, 100, 6912), (8, 160, 2560), (9, 33, 256),
+    (2, 5, 16), (5, 100, 6912), (8, 160, 2560), (7, 3000, 80), (6, 2561, 2560), (9, 33, 256),
     (16, 48, 1024), (17, 31, 192), (24, 64, 2560), (31, 47, 640), (32, 96, 6912),
     (33, 300, 192), (128, 256, 128), (129, 257, 2624), (300, 600, 2560), (256, 520, 64),
     (384, 300, 640), (1000, 512, 2560), (640, 1100, 384),
