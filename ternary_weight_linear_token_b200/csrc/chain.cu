@@ -314,10 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
     // ---------------------------------------------------------- producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int s = 0;
+      int s = 0, slot = 0;
+      uint32_t reuse = 0;  // parity of the slot's release to wait for
       for (; s < P.n_steps; ++s) {
-        const int slot = s % P.slots;
-        if (s >= P.slots && !wait_or_stop(empty + slot, ((s / P.slots) - 1) & 1, stop, P.status)) {
+        if (s >= P.slots && !wait_or_stop(empty + slot, reuse, stop, P.status)) {
           *stop = 1;
           break;
         }
@@ -331,6 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         } else {
           mbar_arrive(full + slot);
         }
+        if (++slot == P.slots) {
+          slot = 0;
+          if (s >= P.slots) reuse ^= 1u;
+        }
       }
       *issued_sh = s;
     }
@@ -338,7 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   } else {
     // ---------------------------------------------------------- consumers
     const unsigned tag = ld_relaxed_u32(P.epoch) + 1u;
-    int consumed = 0;
+    int consumed = 0, slot = 0;
+    uint32_t phase = 0;  // parity of the slot's fill to wait for
     for (int s = 0; s < P.n_steps; ++s) {
       const StepP &d = tab[s];
       const int nw = d.K >> 1;  // input words: two bf16 values each
@@ -432,9 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       }
       consumers_sync();
       // ---- this CTA's rows: warp w takes rows w, w + 16, ... of its range
-      const int slot = s % P.slots;
       // every lane waits (bounded); the warp goes on only if all of them saw the copy land
-      const bool have_w = __all_sync(0xffffffffu, mbar_wait(full + slot, (s / P.slots) & 1, P.status));
+      const bool have_w = __all_sync(0xffffffffu, mbar_wait(full + slot, phase, P.status));
       const int r0 = rr[s].x, rows = rr[s].y - r0;
       if (have_w) {
         consumed = s + 1;
@@ -487,6 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
           st_relaxed_u64(rec, (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(la));
           st_relaxed_u64(rec + 1, (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(ls));
         }
+      }
+      if (++slot == P.slots) {
+        slot = 0;
+        phase ^= 1u;
       }
     }
     if (tid == 0) {

@@ -205,11 +205,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 __device__ __forceinline__ float act_scale(float amax) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(127.0f, amax);
 }
-// clamp(round_half_away(x * s), -127, 127).
+// clamp(round_half_away(x * s), -127, 127), exactly, on the FMA and ALU
+// pipes only (no float-to-int conversion): adding 1.5 * 2^23 to a float of
+// magnitude below 2^22 leaves its nearest integer (ties to even, the IEEE
+// rounding of the add) as the low bits of the sum.  Subtracting it back gives
+// that integer as a float; a tie (the remainder is exactly +-0.5) is then
+// moved away from zero, and the clamped integer is read from the low bits of
+// a second add.  Checked against the plain definition for every float of
+// magnitude up to 128; an in-contract x * s never exceeds 127.00003.
 __device__ __forceinline__ int quant_i8(float x, float s) {
-  float r = roundf(__fmul_rn(x, s));
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
+  const float v = __fmul_rn(x, s);
+  float r = __fsub_rn(__fadd_rn(v, kMagic), kMagic);
+  if (fabsf(__fsub_rn(v, r)) == 0.5f) r = __fadd_rn(v, copysignf(0.5f, v));
   r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return static_cast<int>(r);
+  return static_cast<int>(__float_as_uint(__fadd_rn(r, kMagic)) - 0x4B400000u);
 }
 // y = (float)acc * (gamma / s), then optionally ReLU^2.
 __device__ __forceinline__ float epilogue_value(int acc, float r, bool relu2) {
