@@ -156,6 +156,31 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                    uint32_t flags, bitnet_stream_t stream);
 
 /* ----------------------------------------------------------------------
+ * Y = BitLinear(rms_norm(X)): the weightless RMS normalisation of
+ * bitnet_rms_norm applied to each token of X, rounded to X's dtype, and then
+ * exactly what bitnet_w158a8_matmul computes for that normalised input.  In
+ * a decode stack it joins a layer's input normalisation (the model card's
+ * "subln", 模型详情 -> 架构; no formula on the pages, this is the plain
+ * stand-in) to the projection that reads it, saving one launch per layer.
+ *   X        [M][K] F32 | BF16 (no int8: the normalisation needs the values).
+ *   X_normed [M][K] of X's dtype, or NULL when M <= 8.  Receives the
+ *            normalised input that was quantised (every link can be
+ *            checked).  For M > 8 it is required: the normalisation then
+ *            runs as its own kernel into it, and the matmul reads it.  Must
+ *            not overlap X or Y.
+ * Everything else as bitnet_w158a8_matmul (workspace size from
+ * bitnet_w158a8_matmul_workspace_size with the same arguments).  The
+ * normalisation's fp32 sum may be ordered differently from bitnet_rms_norm's
+ * (not part of the bit-exact contract).
+ * ---------------------------------------------------------------------- */
+bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype, void *X_normed,
+                                            const uint8_t *packed, const float *gamma,
+                                            int64_t M, int64_t N, int64_t K,
+                                            bitnet_epilogue epi, void *Y, bitnet_dtype y_dtype,
+                                            void *workspace, size_t workspace_bytes,
+                                            uint32_t flags, bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
  * bitnet_w158a8_matmul for callers that cannot allocate device memory.
  * (The pages on BitNet b1.58 have no counterpart of this entry point; it is
  * a service of this library.)

@@ -51,6 +51,8 @@ _SIGS = {
     "bitnet_w158a8_matmul": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST, _P, _SZ,
                               C.c_uint32, _P], _ST),
     "bitnet_rms_norm": ([_P, _ST, _I64, _I64, _P, _ST, _P], _ST),
+    "bitnet_rms_norm_w158a8_matmul": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST, _P,
+                                       _SZ, C.c_uint32, _P], _ST),
     "bitnet_w158a8_matmul_noalloc": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST,
                                       C.c_uint32, _P], _ST),
 }
@@ -196,6 +198,43 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
                                   _DTYPE[Y.dtype], _ptr(workspace), ws_bytes,
                                   FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
     _check(st, "bitnet_w158a8_matmul")
+    return Y
+
+
+def bitnet_rms_norm_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                                  X_normed: torch.Tensor | None = None, relu2: bool = False,
+                                  out_dtype: torch.dtype = torch.bfloat16,
+                                  Y: torch.Tensor | None = None,
+                                  workspace: torch.Tensor | None = None,
+                                  weights_static: bool = False, stream=None) -> torch.Tensor:
+    """Y = BitLinear(rms_norm(X)) for fp32/bf16 X [M, K].  X_normed (same
+    dtype and shape as X) receives the normalised input; it may be omitted
+    for M <= 8 and is allocated here otherwise."""
+    _dev(X, "X", (torch.float32, torch.bfloat16))
+    _dev(packed, "packed", (torch.uint8,))
+    _dev(gamma, "gamma", (torch.float32,))
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError(f"packed has {packed.shape[1]} bytes per row, expected K/4 = {K // 4}")
+    if X_normed is None and M > 8:
+        X_normed = torch.empty_like(X)
+    if X_normed is not None:
+        _dev(X_normed, "X_normed", (X.dtype,))
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _dev(Y, "Y", (torch.float32, torch.bfloat16, torch.int32))
+    need = bitnet_w158a8_matmul_workspace_size(M, N, K, X.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.bitnet_rms_norm_w158a8_matmul(_ptr(X), _DTYPE[X.dtype], _ptr(X_normed), _ptr(packed),
+                                           _ptr(gamma), M, N, K,
+                                           EPI_RELU2 if relu2 else EPI_NONE, _ptr(Y),
+                                           _DTYPE[Y.dtype], _ptr(workspace), ws_bytes,
+                                           FLAG_WEIGHTS_STATIC if weights_static else 0,
+                                           _stream(stream))
+    _check(st, "bitnet_rms_norm_w158a8_matmul")
     return Y
 
 

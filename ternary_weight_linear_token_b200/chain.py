@@ -13,8 +13,9 @@ activations vanish within a few layers).
 
 Two ways to run it, both through the C-ABI library on one stream and both
 capturable in a CUDA graph (``capture``):
-  * per launch (default): ``run`` makes one call per projection and one per
-    normalisation, 5 kernels per layer;
+  * per launch (default): ``run`` makes one call per projection, 4 kernels
+    per layer (each layer's QKV call normalises its input itself,
+    ``bitnet_rms_norm_w158a8_matmul``) plus one normalisation at the end;
   * persistent (``persistent=True``): ``run`` makes one call of
     ``bitnet_decode_chain``, one kernel for the whole stack, with the
     normalisation folded into the next layer's QKV projection.
@@ -26,7 +27,8 @@ from __future__ import annotations
 import torch
 
 from . import (bitnet_decode_chain, bitnet_decode_chain_steps, bitnet_decode_chain_workspace_size,
-               bitnet_quantize_weights, bitnet_rms_norm, bitnet_w158a8_matmul)
+               bitnet_quantize_weights, bitnet_rms_norm, bitnet_rms_norm_w158a8_matmul,
+               bitnet_w158a8_matmul)
 
 
 class DecodeChain:
@@ -84,17 +86,22 @@ class DecodeChain:
         if self.persistent:
             bitnet_decode_chain(self._steps, self.x_in, self.workspace, y_norm=self.outs[-1][4])
             return self.outs[-1][4]
-        x = self.x_in
-        for proj, bufs in zip(self.layers, self.outs):
+        for li, (proj, bufs) in enumerate(zip(self.layers, self.outs)):
             qkv, o, up, down = proj
-            self._bl(x, qkv, bufs[0])
+            if li == 0:
+                self._bl(self.x_in, qkv, bufs[0])
+            else:  # the previous layer's normalisation, inside this call
+                prev = self.outs[li - 1]
+                bitnet_rms_norm_w158a8_matmul(prev[3], qkv["packed"], qkv["gamma"],
+                                              X_normed=prev[4], relu2=qkv["relu2"], Y=bufs[0],
+                                              weights_static=self.weights_static)
             q = bufs[0][:, : self.d]          # contiguous for one token
             self._bl(q, o, bufs[1])
             self._bl(bufs[1], up, bufs[2])
             self._bl(bufs[2], down, bufs[3])
-            bitnet_rms_norm(bufs[3], Y=bufs[4])
-            x = bufs[4]
-        return x
+        last = self.outs[-1]
+        bitnet_rms_norm(last[3], Y=last[4])
+        return last[4]
 
     def capture(self) -> torch.cuda.CUDAGraph:
         """Capture one token through the whole stack in a CUDA graph."""
@@ -110,4 +117,4 @@ class DecodeChain:
         return g
 
     def launches_per_token(self) -> int:
-        return 1 if self.persistent else 5 * len(self.layers)
+        return 1 if self.persistent else 4 * len(self.layers) + 1

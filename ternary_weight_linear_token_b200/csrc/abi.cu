@@ -96,6 +96,73 @@ size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
          align256(4 * static_cast<size_t>(M));
 }
 
+// Argument checks of bitnet_w158a8_matmul (and of its normalising variant,
+// which passes s = NULL): BITNET_OK or the status to return.  OK for an
+// empty call whatever the pointers.
+bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
+                           const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
+                           int64_t K, bitnet_epilogue epi, const void *Y, bitnet_dtype y_dtype,
+                           const void *workspace, size_t workspace_bytes, uint32_t flags) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
+    return BITNET_ERR_INVALID_ARG;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32)
+    return BITNET_ERR_INVALID_ARG;
+  if (epi != BITNET_EPI_NONE && epi != BITNET_EPI_RELU2) return BITNET_ERR_INVALID_ARG;
+  if (y_dtype == BITNET_I32 && epi != BITNET_EPI_NONE) return BITNET_ERR_INVALID_ARG;
+  if ((flags & ~BITNET_FLAG_WEIGHTS_STATIC) != 0) return BITNET_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_k(K)) return st;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (X == nullptr || packed == nullptr || gamma == nullptr || Y == nullptr)
+    return BITNET_ERR_INVALID_ARG;
+  if ((x_dtype == BITNET_I8) != (s != nullptr)) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(gamma, 4) ||
+      (s != nullptr && !aligned(s, 4)))
+    return BITNET_ERR_MISALIGNED;
+  if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
+              static_cast<size_t>(M) * N * elem_size(y_dtype)))
+    return BITNET_ERR_INVALID_ARG;
+  const size_t need = matmul_workspace(M, N, K, x_dtype);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  }
+  return BITNET_OK;
+}
+
+// Kernel choice and launches of bitnet_w158a8_matmul once its arguments are
+// checked.
+bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
+                         const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
+                         int64_t K, bool relu2, void *Y, bitnet_dtype y_dtype, void *workspace,
+                         bool wstatic, const LaunchCtx &ctx) {
+  if (rows_supported(M, N, K))
+    return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                 wstatic, false, nullptr, ctx));
+  const bool decode = decode_supported(M, N, K);
+  const bool prefill = !decode && prefill_supported(M, N, K);
+  const int8_t *xq = static_cast<const int8_t *>(X);
+  const float *sq = s;
+  if (x_dtype != BITNET_I8) {
+    // The prefill kernel takes its own quantiser's output in the K order of
+    // its fast weight unpack; the decode and generic kernels want natural order.
+    int8_t *wxq = static_cast<int8_t *>(workspace);
+    float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                          align256(static_cast<size_t>(M) * K));
+    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill, ctx);
+    if (e != cudaSuccess) return BITNET_ERR_CUDA;
+    xq = wxq;
+    sq = ws;
+  }
+  if (decode)
+    return from_cuda(launch_decode(xq, BITNET_I8, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                   wstatic, ctx));
+  if (prefill)
+    return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                    x_dtype != BITNET_I8, ctx));
+  return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
+}
+
 static_assert(kStepRelu2 == BITNET_STEP_RELU2 && kStepNormIn == BITNET_STEP_NORM_IN,
               "step flags");
 static_assert(kChainMaxSteps == BITNET_CHAIN_MAX_STEPS, "chain length");
@@ -123,7 +190,7 @@ bitnet_status check_chain(const bitnet_chain_step *steps, int n_steps) {
 size_t chain_workspace(const bitnet_chain_step *steps, int n_steps) {
   size_t words = 0;
   for (int s = 0; s < n_steps; ++s) words += static_cast<size_t>(chain_xch_words(steps[s].N));
-  return align256(kChainWorkspaceHeader + chain_stats_bytes(n_steps) + 8 * words);
+  return align256(kChainWorkspaceHeader + chain_stats_bytes(n_steps) + kChainReplicas * 8 * words);
 }
 
 }  // namespace
@@ -198,60 +265,46 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                    int64_t N, int64_t K, bitnet_epilogue epi, void *Y,
                                    bitnet_dtype y_dtype, void *workspace, size_t workspace_bytes,
                                    uint32_t flags, bitnet_stream_t stream) {
-  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
-    return BITNET_ERR_INVALID_ARG;
-  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32)
-    return BITNET_ERR_INVALID_ARG;
-  if (epi != BITNET_EPI_NONE && epi != BITNET_EPI_RELU2) return BITNET_ERR_INVALID_ARG;
-  if (y_dtype == BITNET_I32 && epi != BITNET_EPI_NONE) return BITNET_ERR_INVALID_ARG;
-  if ((flags & ~BITNET_FLAG_WEIGHTS_STATIC) != 0) return BITNET_ERR_INVALID_ARG;
-  if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
-  if (bitnet_status st = check_k(K)) return st;
+  if (bitnet_status st = check_matmul(X, x_dtype, s, packed, gamma, M, N, K, epi, Y, y_dtype,
+                                      workspace, workspace_bytes, flags))
+    return st;
   if (M == 0 || N == 0) return BITNET_OK;  // empty: pointers may be NULL
-  if (X == nullptr || packed == nullptr || gamma == nullptr || Y == nullptr)
-    return BITNET_ERR_INVALID_ARG;
-  if ((x_dtype == BITNET_I8) != (s != nullptr)) return BITNET_ERR_INVALID_ARG;
-  if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(gamma, 4) ||
-      (s != nullptr && !aligned(s, 4)))
-    return BITNET_ERR_MISALIGNED;
-  if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
-              static_cast<size_t>(M) * N * elem_size(y_dtype)))
-    return BITNET_ERR_INVALID_ARG;
-  const size_t need = matmul_workspace(M, N, K, x_dtype);
-  if (need > 0) {
-    if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  return run_matmul(X, x_dtype, s, packed, gamma, M, N, K, epi == BITNET_EPI_RELU2, Y, y_dtype,
+                    workspace, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0, ctx);
+}
+
+bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype, void *X_normed,
+                                            const uint8_t *packed, const float *gamma,
+                                            int64_t M, int64_t N, int64_t K,
+                                            bitnet_epilogue epi, void *Y, bitnet_dtype y_dtype,
+                                            void *workspace, size_t workspace_bytes,
+                                            uint32_t flags, bitnet_stream_t stream) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_matmul(X, x_dtype, nullptr, packed, gamma, M, N, K, epi, Y, y_dtype,
+                                      workspace, workspace_bytes, flags))
+    return st;
+  if (M == 0 || N == 0) return BITNET_OK;
+  const size_t x_bytes = static_cast<size_t>(M) * K * elem_size(x_dtype);
+  const bool fused = rows_supported(M, N, K);
+  if (!fused && X_normed == nullptr) return BITNET_ERR_INVALID_ARG;  // needed as the matmul input
+  if (X_normed != nullptr) {
+    if (!aligned(X_normed, 16)) return BITNET_ERR_MISALIGNED;
+    if (overlap(X, x_bytes, X_normed, x_bytes) ||
+        overlap(Y, static_cast<size_t>(M) * N * elem_size(y_dtype), X_normed, x_bytes))
+      return BITNET_ERR_INVALID_ARG;
   }
   LaunchCtx ctx;
   if (bitnet_status st = device_ctx(stream, &ctx)) return st;
   const bool relu2 = epi == BITNET_EPI_RELU2;
   const bool wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
-
-  if (rows_supported(M, N, K))
-    return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                 wstatic, ctx));
-  const bool decode = decode_supported(M, N, K);
-  const bool prefill = !decode && prefill_supported(M, N, K);
-  const int8_t *xq = static_cast<const int8_t *>(X);
-  const float *sq = s;
-  if (x_dtype != BITNET_I8) {
-    // The prefill kernel takes its own quantiser's output in the K order of
-    // its fast weight unpack; the decode and generic kernels want natural order.
-    int8_t *wxq = static_cast<int8_t *>(workspace);
-    float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                          align256(static_cast<size_t>(M) * K));
-    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill, ctx);
-    if (e != cudaSuccess) return BITNET_ERR_CUDA;
-    xq = wxq;
-    sq = ws;
-  }
-  if (decode)
-    return from_cuda(launch_decode(xq, BITNET_I8, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                   wstatic, ctx));
-  if (prefill)
-    return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                    x_dtype != BITNET_I8, ctx));
-  return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
+  if (fused)
+    return from_cuda(launch_rows(X, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                                 wstatic, true, X_normed, ctx));
+  if (launch_rms_norm(X, x_dtype, M, K, X_normed, x_dtype, ctx) != cudaSuccess) return BITNET_ERR_CUDA;
+  return run_matmul(X_normed, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y, y_dtype,
+                    workspace, wstatic, ctx);
 }
 
 bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K, void *Y,

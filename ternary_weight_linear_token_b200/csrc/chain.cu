@@ -69,12 +69,13 @@ struct __align__(8) StepP {
 struct ChainP {
   const uint16_t *x0;
   uint16_t *y_norm;
-  unsigned long long *xch;
-  unsigned long long *stats;  // [n_steps][kMaxCtas][2]: tagged max |y|, sum y^2
+  unsigned long long *xch;    // [kChainReplicas][xch_words]
+  unsigned long long *stats;  // [kChainReplicas][n_steps][kMaxCtas][2]: tagged max |y|, sum y^2
   unsigned int *epoch;
   unsigned int *done;
   int *status;
   int n_steps, ctas, slots, slot_bytes, xq_bytes, ystage_bytes, y_norm_n;
+  int xch_words;  // exchange words of one copy
   StepP steps[kChainMaxSteps];
 };
 
@@ -194,6 +195,7 @@ __device__ __forceinline__ bool poll_stats(const unsigned long long *rec, int ct
       record_status(status, kStatusTimeout);
       return false;
     }
+    __nanosleep(256);  // 148 pollers on the same few lines: leave room for the stores
   }
   a = 0.0f;
   ss = 0.0f;
@@ -342,6 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   } else {
     // ---------------------------------------------------------- consumers
     const unsigned tag = ld_relaxed_u32(P.epoch) + 1u;
+    // the copy of the exchange this CTA reads
+    const unsigned long long *my_stats =
+        P.stats + static_cast<size_t>(blockIdx.x % kChainReplicas) * P.n_steps * kMaxCtas * 2;
+    const unsigned long long *my_xch =
+        P.xch + static_cast<size_t>(blockIdx.x % kChainReplicas) * P.xch_words;
     int consumed = 0, slot = 0;
     uint32_t phase = 0;  // parity of the slot's fill to wait for
     for (int s = 0; s < P.n_steps; ++s) {
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         // computes the scale once; then every thread loads its words
         if (warp == 0 && !*stop) {
           float a, ss;
-          if (poll_stats(P.stats + static_cast<size_t>(s - 1) * kMaxCtas * 2, P.ctas, tag, lane,
+          if (poll_stats(my_stats + static_cast<size_t>(s - 1) * kMaxCtas * 2, P.ctas, tag, lane,
                          a, ss, P.status)) {
             if (lane == 0) {
               float iv = 1.0f;
@@ -415,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         sc = par[0];
         r = par[1];
         inv = par[2];
-        if (!poll_words(P.xch + tab[s - 1].out_off, nw, tid, tag, w, P.status)) {
+        if (!poll_words(my_xch + tab[s - 1].out_off, nw, tid, tag, w, P.status)) {
           *stop = 1;  // acted on at the next step's first barrier
 #pragma unroll
           for (int i = 0; i < kMaxWordsPerThread; ++i) w[i] = 0u;
@@ -465,8 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
           const uint32_t ya = ystage[2 * pl];
           const bool has_b = 2 * pl + 1 < rows;
           const uint32_t yb = has_b ? ystage[2 * pl + 1] : 0u;
-          st_relaxed_u64(P.xch + d.out_off + (r0 >> 1) + pl,
-                         (static_cast<unsigned long long>(tag) << 32) | (yb << 16) | ya);
+          const unsigned long long word = (static_cast<unsigned long long>(tag) << 32) | (yb << 16) | ya;
+#pragma unroll
+          for (int c = 0; c < kChainReplicas; ++c)
+            st_relaxed_u64(P.xch + static_cast<size_t>(c) * P.xch_words + d.out_off + (r0 >> 1) + pl, word);
           if (has_b)
             *reinterpret_cast<uint32_t *>(d.Y + r0 + 2 * pl) = (yb << 16) | ya;
           else
@@ -486,8 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) ls = __fadd_rn(ls, __shfl_xor_sync(0xffffffffu, ls, o));
-        if (lane == 0) {
-          unsigned long long *rec = P.stats + (static_cast<size_t>(s) * kMaxCtas + blockIdx.x) * 2;
+        ls = __shfl_sync(0xffffffffu, ls, 0);  // one value for every copy
+        if (lane < kChainReplicas) {  // lane c writes copy c
+          unsigned long long *rec =
+              P.stats + (static_cast<size_t>(lane) * P.n_steps * kMaxCtas + static_cast<size_t>(s) * kMaxCtas +
+                         blockIdx.x) * 2;
           st_relaxed_u64(rec, (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(la));
           st_relaxed_u64(rec + 1, (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(ls));
         }
@@ -513,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       if (P.y_norm != nullptr) {
         if (warp == 0) {
           float a, ss;
-          if (poll_stats(P.stats + static_cast<size_t>(P.n_steps - 1) * kMaxCtas * 2, P.ctas, tag,
+          if (poll_stats(my_stats + static_cast<size_t>(P.n_steps - 1) * kMaxCtas * 2, P.ctas, tag,
                          lane, a, ss, P.status)) {
             if (lane == 0) par[2] = rms_inv(ss, P.y_norm_n);
           } else {
@@ -523,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         consumers_sync();
         const int nw = P.y_norm_n >> 1;
         uint32_t w[kMaxWordsPerThread];
-        if (!*stop && poll_words(P.xch + tab[P.n_steps - 1].out_off, nw, tid, tag, w, P.status)) {
+        if (!*stop && poll_words(my_xch + tab[P.n_steps - 1].out_off, nw, tid, tag, w, P.status)) {
           const float iv = par[2];
 #pragma unroll
           for (int i = 0; i < kMaxWordsPerThread; ++i) {
@@ -629,6 +641,7 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
     d.out_off = static_cast<int>(off);
     off += chain_xch_words(steps[s].N);
   }
+  p.xch_words = static_cast<int>(off);
   cudaError_t e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(plan.smem));
   if (e != cudaSuccess) return e;

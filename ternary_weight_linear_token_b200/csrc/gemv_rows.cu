@@ -55,10 +55,13 @@ struct RowsParams {
   int xs;        // shared-memory bytes per token row
   int ws;        // shared-memory bytes per weight row
   int weights_static;
+  void *Xn;      // NORM: the normalised input, written by CTA 0 (may be null)
+  int rpw;       // rows per warp in the dot products (1, 2 or 4; > 1 only for M <= 2)
 };
 
-// scales [kMaxTok], gamma/s [kMaxTok], then per-warp maxima [kMaxWarps][kMaxTok]
-constexpr int kHeader = 32 + 32 + kMaxWarps * kMaxTok * 4;
+// scales [kMaxTok], gamma/s [kMaxTok], then per-warp maxima and sums of
+// squares [kMaxWarps][kMaxTok] each
+constexpr int kHeader = 32 + 32 + 2 * kMaxWarps * kMaxTok * 4;
 int x_row_bytes(int K) { return (K + 127) / 128 * 128; }
 int w_row_bytes(int K) { return (K / 4 + 15) / 16 * 16; }
 // One CTA per SM, so that a wide projection never runs a second wave (two
@@ -167,12 +170,37 @@ __device__ __forceinline__ int dot_word(const Unpacked &q, uint4 x, int acc) {
   return acc;
 }
 
-template <int MT, int XK, int YK, bool RELU2>
+// x rounded to the input's precision (the normalised input is stored in it).
+template <int XK>
+__device__ __forceinline__ float round_to_input(float x) {
+  return XK == kBF16 ? __bfloat162float(__float2bfloat16_rn(x)) : x;
+}
+
+// 8 values in the input's precision to memory (16- or 32-byte aligned).
+template <int XK>
+__device__ __forceinline__ void store8(void *X, size_t idx, const float (&v)[8]) {
+  if (XK == kF32) {
+    float4 *p = reinterpret_cast<float4 *>(static_cast<float *>(X) + idx);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      o[h] = (__float_as_uint(v[2 * h]) >> 16) | (__float_as_uint(v[2 * h + 1]) & 0xFFFF0000u);
+    *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(X) + idx) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// NORM: the input is first normalised per token, x / sqrt(mean(x^2) + 1e-6)
+// in fp32, and rounded to its own precision; that is what gets quantised.
+template <int MT, int XK, int YK, bool RELU2, bool NORM>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   float *s_sh = reinterpret_cast<float *>(smem);                 // kMaxTok scales
   float *r_sh = reinterpret_cast<float *>(smem + 32);            // kMaxTok gamma / s
   float *wmax = reinterpret_cast<float *>(smem + 64);            // [kMaxWarps][kMaxTok]
+  float *wss = wmax + kMaxWarps * kMaxTok;                       // [kMaxWarps][kMaxTok]
   uint8_t *xsh = smem + kHeader;
   uint8_t *wsh = xsh + p.M * p.xs;  // the host sizes shared memory for p.M token rows
 
@@ -212,12 +240,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       if (t >= p.M) break;
-      float a = 0.0f;
+      float a = 0.0f, ss = 0.0f;
       if (tid < chunks) {
         float v[8];
         load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
+        for (int e = 0; e < 8; ++e) {
+          a = fmaxf(a, fabsf(v[e]));
+          if (NORM) ss = __fmaf_rn(v[e], v[e], ss);
+        }
         if (t < kCached) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) v0[t < kCached ? t : 0][e] = v[e];
@@ -227,18 +258,37 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
         float v[8];
         load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * c, v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
+        for (int e = 0; e < 8; ++e) {
+          a = fmaxf(a, fabsf(v[e]));
+          if (NORM) ss = __fmaf_rn(v[e], v[e], ss);
+        }
       }
       a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
-      if (lane == 0) wmax[warp * kMaxTok + t] = a;
+      if (NORM) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+      }
+      if (lane == 0) {
+        wmax[warp * kMaxTok + t] = a;
+        if (NORM) wss[warp * kMaxTok + t] = ss;
+      }
     }
     __syncthreads();
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       if (t >= p.M) break;
-      float a = 0.0f;
+      float a = 0.0f, inv = 1.0f;
       for (int i = 0; i < nwarps; ++i) a = fmaxf(a, wmax[i * kMaxTok + t]);
+      if (NORM) {
+        float ss = 0.0f;
+        for (int i = 0; i < nwarps; ++i) ss = __fadd_rn(ss, wss[i * kMaxTok + t]);
+        inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, static_cast<float>(p.K)), 1e-6f)));
+        // rounding x * inv to the input's precision is monotone in |x|: the
+        // max of the normalised values is the normalised max
+        a = round_to_input<XK>(__fmul_rn(a, inv));
+      }
       const float sm = act_scale(a);
+      const bool write_n = NORM && p.Xn != nullptr && blockIdx.x == 0;
       if (tid == blockDim.x - 1) {  // a lane with no activation work in the common case
         s_sh[t] = sm;
         r_sh[t] = __fdiv_rn(*p.gamma, sm);
@@ -252,12 +302,24 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
         } else if (tid < chunks) {
           load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
         }
+        if (NORM && tid < chunks) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = round_to_input<XK>(__fmul_rn(v[e], inv));
+          if (write_n) store8<XK>(p.Xn, static_cast<size_t>(t) * p.K + 8 * tid, v);
+        }
         store_half_group(xrow, tid, v, sm, tid < chunks);
       }
       for (int c0 = blockDim.x; c0 < chunks; c0 += blockDim.x) {  // whole warps iterate together
         const int c = c0 + tid;
         float v[8];
-        if (c < chunks) load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * c, v);
+        if (c < chunks) {
+          load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * c, v);
+          if (NORM) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = round_to_input<XK>(__fmul_rn(v[e], inv));
+            if (write_n) store8<XK>(p.Xn, static_cast<size_t>(t) * p.K + 8 * c, v);
+          }
+        }
         store_half_group(xrow, c, v, sm, c < chunks);
       }
     }
@@ -265,6 +327,63 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
   cp_async_commit_wait();
   __syncthreads();
 
+  // ---- dot products, rpw > 1 (one or two tokens): rpw rows per warp, 32 / rpw
+  // lanes per row.  Lanes at the same word position of different rows read
+  // the same activation bytes (a shared-memory broadcast), so the activations
+  // are read rpw times less often than with one row per warp.
+  if (MT <= 2 && p.rpw > 1) {
+    const int G = 32 / p.rpw, g = lane / G, j = lane % G;
+    for (int rb = warp * p.rpw; rb < rows; rb += nwarps * p.rpw) {
+      const int rl = rb + g;
+      const bool live = rl < rows;
+      const uint32_t *wrow = reinterpret_cast<const uint32_t *>(wsh + (live ? rl : 0) * p.ws);
+      int acc[MT][2];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = 0;
+      int w = j;
+      for (; w + 3 * G < words; w += 4 * G) {  // four words of the row in flight per lane
+        const Unpacked q0 = unpack_word(wrow[w]), q1 = unpack_word(wrow[w + G]);
+        const Unpacked q2 = unpack_word(wrow[w + 2 * G]), q3 = unpack_word(wrow[w + 3 * G]);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (t < p.M) {
+            const uint4 *xr = reinterpret_cast<const uint4 *>(xsh + t * p.xs);
+            const int b0 = dot_word(q0, xr[w], 0), b1 = dot_word(q1, xr[w + G], 0);
+            const int b2 = dot_word(q2, xr[w + 2 * G], 0), b3 = dot_word(q3, xr[w + 3 * G], 0);
+            acc[t][0] += b0 + b2;
+            acc[t][1] += b1 + b3;
+          }
+        }
+      }
+      for (; w < words; w += G) {
+        const Unpacked q = unpack_word(wrow[w]);
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+          if (t < p.M)
+            acc[t][0] = dot_word(q, *reinterpret_cast<const uint4 *>(xsh + t * p.xs + 16 * w), acc[t][0]);
+      }
+      int res = 0;
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        int v = acc[t][0] + acc[t][1];
+        for (int o = G >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (j == t) res = v;
+      }
+      if (live && j < p.M) {
+        const size_t o = static_cast<size_t>(j) * p.N + n0 + rl;
+        if (YK == kI32) {
+          static_cast<int *>(p.Y)[o] = res;
+        } else {
+          const float y = epilogue_value(res, r_sh[j], RELU2);
+          if (YK == kF32)
+            static_cast<float *>(p.Y)[o] = y;
+          else
+            static_cast<__nv_bfloat16 *>(p.Y)[o] = __float2bfloat16_rn(y);
+        }
+      }
+    }
+    return;
+  }
   // ---- dot products: warp w takes rows w, w + nwarps, ... of the CTA's range
   for (int rl = warp; rl < rows; rl += nwarps) {
     const uint32_t *wrow = reinterpret_cast<const uint32_t *>(wsh + rl * p.ws);
@@ -272,6 +391,22 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
 #pragma unroll
     for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = 0;
     int w = lane;
+    if (MT <= 2) {  // four words of the row in flight per lane
+      for (; w + 96 < words; w += 128) {
+        const Unpacked q0 = unpack_word(wrow[w]), q1 = unpack_word(wrow[w + 32]);
+        const Unpacked q2 = unpack_word(wrow[w + 64]), q3 = unpack_word(wrow[w + 96]);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (t < p.M) {
+            const uint4 *xr = reinterpret_cast<const uint4 *>(xsh + t * p.xs);
+            const int b0 = dot_word(q0, xr[w], 0), b1 = dot_word(q1, xr[w + 32], 0);
+            const int b2 = dot_word(q2, xr[w + 64], 0), b3 = dot_word(q3, xr[w + 96], 0);
+            acc[t][0] += b0 + b2;
+            acc[t][1] += b1 + b3;
+          }
+        }
+      }
+    }
     for (; w + 32 < words; w += 64) {
       const Unpacked qa = unpack_word(wrow[w]), qb = unpack_word(wrow[w + 32]);
 #pragma unroll
@@ -310,36 +445,50 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
   }
 }
 
-template <int MT, int XK, int YK, bool RELU2>
+template <int MT, int XK, int YK, bool RELU2, bool NORM>
 cudaError_t launch_t(const RowsParams &p, size_t smem, const LaunchCtx &ctx) {
-  auto kern = rows_kernel<MT, XK, YK, RELU2>;
+  auto kern = rows_kernel<MT, XK, YK, RELU2, NORM>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
+  // At most half the SM's registers per CTA, so that the next call's CTA can
+  // be resident (and prefetch its weights) while this one still runs.
+  static const int max_warps = [&] {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, kern) != cudaSuccess || a.numRegs <= 0) return 16;
+    const int regs = (a.numRegs + 7) / 8 * 8;  // allocation granularity
+    const int w = 32768 / (32 * regs);
+    return w < 2 ? 2 : (w > kMaxWarps ? kMaxWarps : w);
+  }();
   const int rpc = rows_per_cta(p.N, p.ctas);
-  const int warps = rpc < kMaxWarps ? rpc : kMaxWarps;
-  // an even warp count keeps the activation half-group pairs in whole warps
+  const int want = (rpc + p.rpw - 1) / p.rpw;
+  const int warps = want < max_warps ? want : max_warps;
   return launch_k(kern, dim3(static_cast<unsigned>(p.ctas)), dim3(32 * (warps < 2 ? 2 : warps)),
                   smem, ctx, p);
 }
 
-template <int MT, int XK>
+template <int MT, int XK, bool NORM>
 cudaError_t dispatch_y(const RowsParams &p, size_t smem, int y_kind, bool relu2,
                        const LaunchCtx &ctx) {
-  if (y_kind == kI32) return launch_t<MT, XK, kI32, false>(p, smem, ctx);
+  if (y_kind == kI32) return launch_t<MT, XK, kI32, false, NORM>(p, smem, ctx);
   if (y_kind == kF32)
-    return relu2 ? launch_t<MT, XK, kF32, true>(p, smem, ctx) : launch_t<MT, XK, kF32, false>(p, smem, ctx);
-  return relu2 ? launch_t<MT, XK, kBF16, true>(p, smem, ctx) : launch_t<MT, XK, kBF16, false>(p, smem, ctx);
+    return relu2 ? launch_t<MT, XK, kF32, true, NORM>(p, smem, ctx)
+                 : launch_t<MT, XK, kF32, false, NORM>(p, smem, ctx);
+  return relu2 ? launch_t<MT, XK, kBF16, true, NORM>(p, smem, ctx)
+               : launch_t<MT, XK, kBF16, false, NORM>(p, smem, ctx);
 }
 
 template <int MT>
 cudaError_t dispatch_x(const RowsParams &p, size_t smem, int x_kind, int y_kind, bool relu2,
-                       const LaunchCtx &ctx) {
-  if (x_kind == kI8) return dispatch_y<MT, kI8>(p, smem, y_kind, relu2, ctx);
-  if (x_kind == kF32) return dispatch_y<MT, kF32>(p, smem, y_kind, relu2, ctx);
-  return dispatch_y<MT, kBF16>(p, smem, y_kind, relu2, ctx);
+                       bool norm, const LaunchCtx &ctx) {
+  if (x_kind == kI8) return dispatch_y<MT, kI8, false>(p, smem, y_kind, relu2, ctx);
+  if (x_kind == kF32)
+    return norm ? dispatch_y<MT, kF32, true>(p, smem, y_kind, relu2, ctx)
+                : dispatch_y<MT, kF32, false>(p, smem, y_kind, relu2, ctx);
+  return norm ? dispatch_y<MT, kBF16, true>(p, smem, y_kind, relu2, ctx)
+              : dispatch_y<MT, kBF16, false>(p, smem, y_kind, relu2, ctx);
 }
 
 }  // namespace
@@ -353,7 +502,9 @@ bool rows_supported(int64_t M, int64_t N, int64_t K) {
 
 cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t *packed,
                         const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2, void *Y,
-                        int y_kind, bool weights_static, const LaunchCtx &ctx) {
+                        int y_kind, bool weights_static, bool norm, void *Xn,
+                        const LaunchCtx &ctx) {
+  if (norm && x_kind == kI8) return cudaErrorInvalidValue;
   RowsParams p;
   p.X = X;
   p.s_in = s;
@@ -367,12 +518,20 @@ cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t
   p.xs = x_row_bytes(static_cast<int>(K));
   p.ws = w_row_bytes(static_cast<int>(K));
   p.weights_static = weights_static ? 1 : 0;
+  p.Xn = Xn;
+  // Two rows per warp for one or two tokens when a CTA owns many rows: half
+  // the activation re-reads of the dot products, for twice the words per
+  // lane and half the warps.  Measured per M = 1 call (dependent calls, bf16):
+  // N = 3840 (26 rows per CTA) 3.71 -> 3.09 us and N = 6912 (47 rows) 4.53 ->
+  // 4.16 us, but N = 2560 (18 rows) 2.51 -> 3.53 us, where too few warps are
+  // left for the activation prologue.
+  p.rpw = (M <= 2 && rows_per_cta(N, p.ctas) >= 24) ? 2 : 1;
   const size_t smem = rows_smem(static_cast<int>(M), static_cast<int>(K), rows_per_cta(N, p.ctas));
   if (smem > static_cast<size_t>(kSmemLimit)) return cudaErrorInvalidValue;
-  if (M == 1) return dispatch_x<1>(p, smem, x_kind, y_kind, relu2, ctx);
-  if (M == 2) return dispatch_x<2>(p, smem, x_kind, y_kind, relu2, ctx);
-  if (M <= 4) return dispatch_x<4>(p, smem, x_kind, y_kind, relu2, ctx);
-  return dispatch_x<8>(p, smem, x_kind, y_kind, relu2, ctx);
+  if (M == 1) return dispatch_x<1>(p, smem, x_kind, y_kind, relu2, norm, ctx);
+  if (M == 2) return dispatch_x<2>(p, smem, x_kind, y_kind, relu2, norm, ctx);
+  if (M <= 4) return dispatch_x<4>(p, smem, x_kind, y_kind, relu2, norm, ctx);
+  return dispatch_x<8>(p, smem, x_kind, y_kind, relu2, norm, ctx);
 }
 
 }  // namespace bitnet

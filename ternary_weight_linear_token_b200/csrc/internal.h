@@ -31,11 +31,14 @@ cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K,
 cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
                             const LaunchCtx &ctx);
 
-// gemv_rows.cu: lowest-latency kernel for 1 <= M <= 4 tokens, any K % 16 == 0.
+// gemv_rows.cu: lowest-latency kernel for 1 <= M <= 8 tokens, any K % 16 == 0.
+// norm (float input only): RMS-normalise each token first; CTA 0 writes the
+// normalised input to Xn when it is not null.
 bool rows_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t *packed,
                         const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2, void *Y,
-                        int y_kind, bool weights_static, const LaunchCtx &ctx);
+                        int y_kind, bool weights_static, bool norm, void *Xn,
+                        const LaunchCtx &ctx);
 
 // gemv_decode.cu: fused decode kernel, M <= 32, K % 64 == 0.
 bool decode_supported(int64_t M, int64_t N, int64_t K);
@@ -62,9 +65,14 @@ constexpr int kStepRelu2 = 1;
 constexpr int kStepNormIn = 2;
 constexpr size_t kChainWorkspaceHeader = 256;  // launch counter, finished-CTA counter
 constexpr int kChainMaxCtas = 256;              // CTAs of one chain launch, at most
-// Per-step, per-CTA records (two tagged 64-bit words: max |y|, sum y^2),
-// after the header; they double as the CTA's "outputs are out" flag.
-inline size_t chain_stats_bytes(int n_steps) { return static_cast<size_t>(n_steps) * kChainMaxCtas * 16; }
+// Copies of everything the CTAs exchange (CTA c reads copy c % kChainReplicas),
+// so that fewer SMs poll and load the same L2 lines.
+constexpr int kChainReplicas = 4;
+// Per-step, per-CTA records (two tagged 64-bit words: max |y|, sum y^2), one
+// set per copy, after the header; they double as the CTA's "outputs are out" flag.
+inline size_t chain_stats_bytes(int n_steps) {
+  return static_cast<size_t>(kChainReplicas) * n_steps * kChainMaxCtas * 16;
+}
 struct ChainStep {
   const uint8_t *packed;
   const float *gamma;

@@ -7,7 +7,9 @@
 // warp shuffles (max is order-independent, so it is exact), then
 // s = 127 / amax and xq = clamp(round_half_away(x * s), -127, 127).  The
 // second pass re-reads the row, which is still in L1.  16 elements (one
-// 16-byte int8 output chunk) per lane-step; K % 16 == 0.
+// 16-byte int8 output chunk) per lane-step, four steps per lane in flight at
+// a time (a K = 2560 row is two dependent rounds of loads, not five);
+// K % 16 == 0.
 #include "common.cuh"
 #include "internal.h"
 
@@ -63,26 +65,77 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
   if (m < M) {
+    // 16-element steps per lane per round: the raw words stay in registers
+    constexpr int kInFlight = KIND == kF32 ? 2 : 4;
+    constexpr int kWords = KIND == kF32 ? 4 : 2;  // uint4 per 16 elements
     const int64_t chunks = K / 16;
-    float amax = 0.0f;
-    for (int64_t c = lane; c < chunks; c += 32) {
-      float v[16];
-      load16<KIND>(X, m * K + 16 * c, v);
+    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(X) +
+                                                      m * K * (KIND == kF32 ? 4 : 2));
+    // max |x| on the bit patterns: |x| of a float (or of a bf16) orders as an unsigned integer
+    uint32_t amax_bits = 0;
+    for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kInFlight) {
+      uint4 raw[kInFlight][kWords];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      for (int i = 0; i < kInFlight; ++i)
+        if (c0 + 32 * i < chunks) {
+#pragma unroll
+          for (int j = 0; j < kWords; ++j) raw[i][j] = row[(c0 + 32 * i) * kWords + j];
+        }
+#pragma unroll
+      for (int i = 0; i < kInFlight; ++i)
+        if (c0 + 32 * i < chunks) {
+#pragma unroll
+          for (int j = 0; j < kWords; ++j) {
+            const uint32_t w[4] = {raw[i][j].x, raw[i][j].y, raw[i][j].z, raw[i][j].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              if (KIND == kF32) {
+                amax_bits = max(amax_bits, w[h] & 0x7FFFFFFFu);
+              } else {
+                amax_bits = max(amax_bits, (w[h] & 0x7FFFu) << 16);
+                amax_bits = max(amax_bits, w[h] & 0x7FFF0000u);
+              }
+            }
+          }
+        }
     }
-    amax = warp_max(amax);
+    const float amax = warp_max(__uint_as_float(amax_bits));
     const float sm = act_scale(amax);
-    for (int64_t c = lane; c < chunks; c += 32) {
-      float v[16];
-      load16<KIND>(X, m * K + 16 * c, v);
-      int q[16];
+    for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kInFlight) {
+      uint4 raw[kInFlight][kWords];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
-      *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) =
-          PERM ? pack_permuted(q)
-               : make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
-                            pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
+      for (int i = 0; i < kInFlight; ++i)
+        if (c0 + 32 * i < chunks) {
+#pragma unroll
+          for (int j = 0; j < kWords; ++j) raw[i][j] = row[(c0 + 32 * i) * kWords + j];
+        }
+#pragma unroll
+      for (int i = 0; i < kInFlight; ++i) {
+        const int64_t c = c0 + 32 * i;
+        if (c < chunks) {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < kWords; ++j) {
+            const uint32_t w[4] = {raw[i][j].x, raw[i][j].y, raw[i][j].z, raw[i][j].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              if (KIND == kF32) {
+                v[4 * j + h] = __uint_as_float(w[h]);
+              } else {
+                v[8 * j + 2 * h] = __uint_as_float(w[h] << 16);
+                v[8 * j + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+              }
+            }
+          }
+          int q[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
+          *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) =
+              PERM ? pack_permuted(q)
+                   : make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                                pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
+        }
+      }
     }
     if (lane == 0) s[m] = sm;
   }

@@ -167,10 +167,28 @@ def test_decode_chain_rejects_bad_arguments(tw):
 def test_decode_chain_workspace_size(tw):
     f = tw.lib.bitnet_decode_chain_workspace_size
     layer = [(3840, 2560), (2560, 2560), (6912, 2560), (2560, 6912)]
-    # 256-byte header, one 16-byte record per CTA (up to 256) per step, then
-    # one 8-byte word per two outputs of every step
+    # 256-byte header; then 4 copies of: one 16-byte record per CTA (up to
+    # 256) per step; then 4 copies of: one 8-byte word per two outputs of
+    # every step
     words = sum((n + 1) // 2 for n, _ in layer)
-    assert f(chain(tw, layer), 4) == (256 + 4 * 4096 + 8 * words + 255) // 256 * 256
-    assert f(chain(tw, [(333, 64)]), 1) == 5888      # 256 + 4096 + 8 * 167 = 5688, rounded up
+    assert f(chain(tw, layer), 4) == (256 + 4 * 4 * 4096 + 4 * 8 * words + 255) // 256 * 256
+    assert f(chain(tw, [(333, 64)]), 1) == 22016     # 256 + 16384 + 5344 = 21984, rounded up
     assert f(chain(tw, [(64, 40)]), 1) == 0          # invalid descriptors
     assert f(chain(tw, layer * 30), 120) > 0
+
+
+def test_rms_norm_matmul_rejects_bad_arguments(tw):
+    f = tw.lib.bitnet_rms_norm_w158a8_matmul
+
+    def call(X=A, xd=1, Xn=None, P=B, g=G, M=4, N=8, K=64, epi=0, Y=Cc, yd=1, ws=None, wsb=0,
+             flags=0):
+        return f(X, xd, Xn, P, g, M, N, K, epi, Y, yd, ws, wsb, flags, None)
+
+    assert call(xd=2) == tw.ERR_INVALID_ARG                       # int8 input
+    assert call(yd=2) == tw.ERR_INVALID_ARG
+    assert call(K=40) == tw.ERR_UNSUPPORTED_SHAPE
+    assert call(M=9, ws=WS, wsb=1 << 20) == tw.ERR_INVALID_ARG    # M > 8 needs X_normed
+    assert call(Xn=MIS) == tw.ERR_MISALIGNED
+    assert call(Xn=C.c_void_p(0x10000000)) == tw.ERR_INVALID_ARG  # X_normed overlapping X
+    assert call(Xn=C.c_void_p(0x30000000)) == tw.ERR_INVALID_ARG  # X_normed overlapping Y
+    assert call(M=0) == tw.OK

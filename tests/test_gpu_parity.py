@@ -317,6 +317,77 @@ def test_chain_link_by_link(tw):
     assert np.array_equal(bf16_bits_of(chain.outs[-1][4]), eager)
 
 
+def test_quantize_act_rounding_near_every_tie(tw):
+    """Every row has max |x| = 127, so s = 127 / 127 = 1 exactly and x * s = x:
+    the kernel's rounding is seen directly.  Rows hold every tie k + 0.5
+    (k = -127..126) with the 64 floats on each side of it, plus uniform
+    values; xq must equal the oracle's round-half-away-from-zero bit for bit."""
+    vals = []
+    for k in range(-127, 127):
+        t = np.float32(k + 0.5)
+        lo = hi = t
+        vals.append(t)
+        for _ in range(64):
+            lo = np.nextafter(lo, np.float32(-np.inf), dtype=np.float32)
+            hi = np.nextafter(hi, np.float32(np.inf), dtype=np.float32)
+            vals += [lo, hi]
+    vals = np.array(vals, dtype=np.float32)
+    vals = vals[np.abs(vals) <= 127.0]
+    rng = np.random.default_rng(5)
+    K = 4096
+    body = np.concatenate([vals, rng.uniform(-127, 127, 64 * K).astype(np.float32)])
+    M = (body.size + K - 2) // (K - 1)
+    body = np.resize(body, M * (K - 1)).reshape(M, K - 1)
+    x = np.concatenate([np.full((M, 1), 127.0, np.float32), body], axis=1)
+    xq, sc = tw.bitnet_quantize_act(f32_t(x))
+    torch.cuda.synchronize()
+    wq, ws = ref.quantize_act(x)
+    assert np.all(ws == np.float32(1.0)) and np.array_equal(np_of(sc), ws)
+    assert np.array_equal(np_of(xq), wq)
+
+
+# (M, N, K, input dtype, ReLU^2): one-launch fused path for M <= 8, a
+# normalisation kernel and then the matmul for larger M
+NORM_SHAPES = [(1, 2560, 2560, "bf16", False), (1, 3840, 2560, "bf16", False),
+               (3, 640, 2560, "f32", True), (8, 300, 320, "bf16", True), (5, 77, 48, "f32", False),
+               (2, 6912, 2560, "bf16", True), (9, 200, 512, "bf16", False),
+               (33, 128, 256, "f32", True)]
+
+
+@pytest.mark.parametrize("M,N,K,dt,relu2", NORM_SHAPES)
+def test_rms_norm_matmul(tw, M, N, K, dt, relu2):
+    """Y = BitLinear(rms_norm(X)): the normalised input against the oracle's
+    normalisation (outside the bit-exact contract: 1 bf16 ulp, or 4e-6
+    relative in fp32), and Y bit-exact against the oracle's BitLinear of the
+    kernel's own normalised input."""
+    rng = np.random.default_rng(M * 131 + N + K)
+    W = synth.latent_weights(rng, N, K)
+    x = (3.0 * rng.standard_t(3, (M, K))).astype(np.float32)
+    X, xf = as_x(x, dt)
+    pd, gd = tw.bitnet_quantize_weights(f32_t(W))
+    po, go = ref.quantize_weights(W)
+    Xn = torch.empty_like(X)
+    ydt = torch.float32 if dt == "f32" else torch.bfloat16
+    Y = tw.bitnet_rms_norm_w158a8_matmul(X, pd, gd, X_normed=Xn, relu2=relu2, out_dtype=ydt)
+    torch.cuda.synchronize()
+    want_n = ref.rms_norm(xf)
+    if dt == "bf16":
+        got_n = bf16_bits_of(Xn)
+        assert_bf16_within_ulp(got_n, ref.to_bf16(want_n), 1)
+        want = ref.to_bf16(ref.bitlinear(synth.bf16_bits_to_f32(got_n), po, go, N, relu2=relu2)["y"])
+        assert np.array_equal(bf16_bits_of(Y), want)
+    else:
+        got_n = np_of(Xn)
+        assert_f32_close(got_n, want_n, rel=4e-6)
+        want = ref.bitlinear(got_n, po, go, N, relu2=relu2)["y"]
+        assert_f32_close(np_of(Y), want)
+    if M <= 8:  # without X_normed: the same result
+        Y2 = tw.bitnet_rms_norm_w158a8_matmul(X, pd, gd, relu2=relu2, out_dtype=ydt)
+        torch.cuda.synchronize()
+        assert torch.equal(Y2, Y)
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
 def test_repeatable(tw):
     d = synth.config_inputs("sweep", M=8, proj=0)
     pd, gd = tw.bitnet_quantize_weights(f32_t(d["W"]))
