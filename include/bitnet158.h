@@ -144,8 +144,10 @@ bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M
  *            bytes (may be NULL when that is 0).  Contents on entry don't
  *            matter; the call may overwrite all of it.
  *   flags    0 or BITNET_FLAG_WEIGHTS_STATIC.
- * Decode-sized calls (M <= 32) run one fused kernel; larger M runs the
- * activation quantiser into the workspace and then the tensor-core kernel.
+ * Up to 3 tokens (8 when K % 64 != 0) run one fused kernel and need no
+ * workspace.  Otherwise fp32/bf16 input is first quantised into the
+ * workspace by the activation quantiser; then 4..32 tokens run an int8
+ * mma.sync kernel and larger M the tcgen05 tensor-core kernel.
  * ---------------------------------------------------------------------- */
 size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype);
 
@@ -168,8 +170,9 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
  *            checked).  For M > 8 it is required: the normalisation then
  *            runs as its own kernel into it, and the matmul reads it.  Must
  *            not overlap X or Y.
- * Everything else as bitnet_w158a8_matmul (workspace size from
- * bitnet_w158a8_matmul_workspace_size with the same arguments).  The
+ * Everything else as bitnet_w158a8_matmul.  Workspace: none when M <= 8 and
+ * K % 16 == 0 fit the fused kernel, otherwise
+ * bitnet_w158a8_matmul_workspace_size(M, N, K, x_dtype) bytes.  The
  * normalisation's fp32 sum may be ordered differently from bitnet_rms_norm's
  * (not part of the bit-exact contract).
  * ---------------------------------------------------------------------- */
@@ -196,7 +199,7 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
  *   - A call whose scratch need, bitnet_w158a8_matmul_workspace_size(M, N,
  *     K, x_dtype), is larger than BITNET_STATIC_SCRATCH_BYTES returns
  *     BITNET_ERR_WORKSPACE and launches nothing.  The need is 0 for int8
- *     input and for decode sizes, and about M*K bytes otherwise.
+ *     input and for up to 3 tokens, and about M*K bytes otherwise.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

@@ -3,10 +3,13 @@
 //
 // Every check runs before any CUDA call, so a rejected call has no side
 // effect and needs no GPU.  Paths of bitnet_w158a8_matmul:
-//   rows     M <= 8: one fused low-latency kernel (warp per output feature,
-//            dp4a; activation quantisation inside).
-//   decode   9 <= M <= 32, K % 64 == 0: bitnet_quantize_act into the
-//            workspace (unless xq is given), then the int8 mma.sync kernel.
+//   rows     M <= 3 (M <= 8 when K % 64 != 0): one fused low-latency kernel
+//            (warp per output feature, dp4a; activation quantisation inside).
+//   mmv      4 <= M <= 32, K % 64 == 0, fp32/bf16 input: bitnet_quantize_act
+//            into the workspace, then the int8 mma.sync kernel with the
+//            tokens as the A operand.
+//   decode   9 <= M <= 32, K % 64 == 0, int8 input (natural K order): the
+//            int8 mma.sync kernel with the weights as the A operand.
 //   prefill  otherwise, K % 64 == 0: bitnet_quantize_act into the workspace
 //            (unless xq is given), then the tcgen05 tensor-core kernel.
 //   generic  K % 64 != 0: quantise into the workspace, then the dp4a kernel.
@@ -86,12 +89,26 @@ bitnet_status check_k(int64_t K) {
 
 bitnet_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
 
+// From here on quantise-then-mma.sync beats the fused dp4a kernel (measured
+// per call on the decode projections, dependent calls: at M = 2 the fused
+// kernel, 3.7 us for 2560 x 2560 against about 5.5 us; at M = 4 the
+// mma.sync path, which stays near 5.5 us up to M = 32).
+constexpr int64_t kMmvMinM = 4;
+
+// The fused one-launch kernel serves this call (int8 input in natural K
+// order always takes it when it can: the mma.sync kernel wants the
+// quantiser's unpack order).
+bool use_rows(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
+  return rows_supported(M, N, K) &&
+         (x_dtype == BITNET_I8 || M < kMmvMinM || !mmv_supported(M, N, K));
+}
+
 // Scratch the matmul needs: int8 xq [M][K] and fp32 s [M] whenever the
-// activation quantiser runs as its own kernel (decode, prefill and generic
-// paths with float input).  Pure arithmetic: no CUDA call.
+// activation quantiser runs as its own kernel (every path but the fused
+// one, with float input).  Pure arithmetic: no CUDA call.
 size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
   if (M <= 0 || N <= 0 || K <= 0 || x_dtype == BITNET_I8) return 0;
-  if (rows_supported(M, N, K)) return 0;
+  if (use_rows(M, N, K, x_dtype)) return 0;
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
          align256(4 * static_cast<size_t>(M));
 }
@@ -102,7 +119,8 @@ size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
 bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                            const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
                            int64_t K, bitnet_epilogue epi, const void *Y, bitnet_dtype y_dtype,
-                           const void *workspace, size_t workspace_bytes, uint32_t flags) {
+                           const void *workspace, size_t workspace_bytes, uint32_t flags,
+                           bool norm_in) {
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
     return BITNET_ERR_INVALID_ARG;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32)
@@ -122,7 +140,8 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
   if (overlap(X, static_cast<size_t>(M) * K * elem_size(x_dtype), Y,
               static_cast<size_t>(M) * N * elem_size(y_dtype)))
     return BITNET_ERR_INVALID_ARG;
-  const size_t need = matmul_workspace(M, N, K, x_dtype);
+  // the normalising variant runs the fused kernel, with no scratch, whenever it can
+  const size_t need = norm_in && rows_supported(M, N, K) ? 0 : matmul_workspace(M, N, K, x_dtype);
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return BITNET_ERR_MISALIGNED;
@@ -136,30 +155,34 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                          const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
                          int64_t K, bool relu2, void *Y, bitnet_dtype y_dtype, void *workspace,
                          bool wstatic, const LaunchCtx &ctx) {
-  if (rows_supported(M, N, K))
+  if (use_rows(M, N, K, x_dtype))
     return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                  wstatic, false, nullptr, ctx));
-  const bool decode = decode_supported(M, N, K);
-  const bool prefill = !decode && prefill_supported(M, N, K);
+  const bool from_float = x_dtype != BITNET_I8;
+  const bool mmv = from_float && mmv_supported(M, N, K);
+  const bool decode = !from_float && decode_supported(M, N, K);  // caller's int8, 9..32 tokens
+  const bool prefill = !mmv && !decode && prefill_supported(M, N, K);
   const int8_t *xq = static_cast<const int8_t *>(X);
   const float *sq = s;
-  if (x_dtype != BITNET_I8) {
-    // The prefill kernel takes its own quantiser's output in the K order of
-    // its fast weight unpack; the decode and generic kernels want natural order.
+  if (from_float) {
+    // The prefill and mmv kernels take the quantiser's output in the K order
+    // of their fast weight unpack; the generic kernel wants natural order.
     int8_t *wxq = static_cast<int8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                           align256(static_cast<size_t>(M) * K));
-    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill, ctx);
+    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill || mmv, ctx);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     xq = wxq;
     sq = ws;
   }
+  if (mmv)
+    return from_cuda(launch_mmv(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, wstatic, ctx));
   if (decode)
     return from_cuda(launch_decode(xq, BITNET_I8, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                    wstatic, ctx));
   if (prefill)
     return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                    x_dtype != BITNET_I8, ctx));
+                                    from_float, ctx));
   return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
 }
 
@@ -266,7 +289,7 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                    bitnet_dtype y_dtype, void *workspace, size_t workspace_bytes,
                                    uint32_t flags, bitnet_stream_t stream) {
   if (bitnet_status st = check_matmul(X, x_dtype, s, packed, gamma, M, N, K, epi, Y, y_dtype,
-                                      workspace, workspace_bytes, flags))
+                                      workspace, workspace_bytes, flags, false))
     return st;
   if (M == 0 || N == 0) return BITNET_OK;  // empty: pointers may be NULL
   LaunchCtx ctx;
@@ -283,11 +306,11 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
                                             uint32_t flags, bitnet_stream_t stream) {
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
   if (bitnet_status st = check_matmul(X, x_dtype, nullptr, packed, gamma, M, N, K, epi, Y, y_dtype,
-                                      workspace, workspace_bytes, flags))
+                                      workspace, workspace_bytes, flags, true))
     return st;
   if (M == 0 || N == 0) return BITNET_OK;
   const size_t x_bytes = static_cast<size_t>(M) * K * elem_size(x_dtype);
-  const bool fused = rows_supported(M, N, K);
+  const bool fused = rows_supported(M, N, K);  // the NORM variant of the fused kernel, M <= 8
   if (!fused && X_normed == nullptr) return BITNET_ERR_INVALID_ARG;  // needed as the matmul input
   if (X_normed != nullptr) {
     if (!aligned(X_normed, 16)) return BITNET_ERR_MISALIGNED;

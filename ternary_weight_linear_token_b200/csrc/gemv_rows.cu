@@ -107,6 +107,42 @@ __device__ __forceinline__ void start_weight_copy(const RowsParams &p, int n0, i
   }
 }
 
+// 8 consecutive activations (16- or 32-byte aligned) as raw words, and
+// their fp32 values.
+template <int KIND>
+struct Raw8 {
+  uint4 u[KIND == kF32 ? 2 : 1];
+};
+template <int KIND>
+__device__ __forceinline__ Raw8<KIND> load_raw8(const void *X, size_t idx) {
+  Raw8<KIND> r;
+  if (KIND == kF32) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const float *>(X) + idx);
+    r.u[0] = p[0];
+    r.u[KIND == kF32 ? 1 : 0] = p[1];
+  } else {
+    r.u[0] = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(X) + idx);
+  }
+  return r;
+}
+template <int KIND>
+__device__ __forceinline__ void raw8_to_float(const Raw8<KIND> &r, float (&v)[8]) {
+  if (KIND == kF32) {
+    const uint32_t w[8] = {r.u[0].x, r.u[0].y, r.u[0].z, r.u[0].w, r.u[KIND == kF32 ? 1 : 0].x,
+                           r.u[KIND == kF32 ? 1 : 0].y, r.u[KIND == kF32 ? 1 : 0].z,
+                           r.u[KIND == kF32 ? 1 : 0].w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(w[e]);
+  } else {
+    const uint32_t w[4] = {r.u[0].x, r.u[0].y, r.u[0].z, r.u[0].w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      v[2 * h] = __uint_as_float(w[h] << 16);
+      v[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+    }
+  }
+}
+
 // 8 consecutive activations (16- or 32-byte aligned) as fp32.
 template <int KIND>
 __device__ __forceinline__ void load8(const void *X, size_t idx, float (&v)[8]) {
@@ -194,8 +230,12 @@ __device__ __forceinline__ void store8(void *X, size_t idx, const float (&v)[8])
 
 // NORM: the input is first normalised per token, x / sqrt(mean(x^2) + 1e-6)
 // in fp32, and rounded to its own precision; that is what gets quantised.
+// Warps per CTA at most: four or more tokens need more registers per thread.
+template <int MT>
+constexpr int warp_cap() { return MT >= 4 ? kMaxWarps / 2 : kMaxWarps; }
+
 template <int MT, int XK, int YK, bool RELU2, bool NORM>
-__global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParams p) {
+__global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const RowsParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   float *s_sh = reinterpret_cast<float *>(smem);                 // kMaxTok scales
   float *r_sh = reinterpret_cast<float *>(smem + 32);            // kMaxTok gamma / s
@@ -235,23 +275,28 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
     }
   } else {
     const int chunks = p.K / 8;
-    constexpr int kCached = MT <= 2 ? MT : 1;  // tokens whose first 8 elements stay in registers
-    float v0[kCached][8];
+    // Tokens whose first 8 elements (per thread) are loaded up front, all at
+    // once, and stay in registers for both passes: the loads of different
+    // tokens are then in flight together instead of one token after another.
+    constexpr int kCached = XK == kF32 ? (MT < 4 ? MT : 4) : MT;
+    Raw8<XK> c0[kCached];
+#pragma unroll
+    for (int t = 0; t < kCached; ++t)
+      if (t < p.M && tid < chunks) c0[t] = load_raw8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid);
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       if (t >= p.M) break;
       float a = 0.0f, ss = 0.0f;
       if (tid < chunks) {
         float v[8];
-        load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
+        if (t < kCached)
+          raw8_to_float<XK>(c0[t < kCached ? t : 0], v);
+        else
+          load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           a = fmaxf(a, fabsf(v[e]));
           if (NORM) ss = __fmaf_rn(v[e], v[e], ss);
-        }
-        if (t < kCached) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v0[t < kCached ? t : 0][e] = v[e];
         }
       }
       for (int c = tid + blockDim.x; c < chunks; c += blockDim.x) {
@@ -297,8 +342,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) rows_kernel(const RowsParam
       {
         float v[8];
         if (t < kCached) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = v0[t < kCached ? t : 0][e];
+          if (tid < chunks) raw8_to_float<XK>(c0[t < kCached ? t : 0], v);
         } else if (tid < chunks) {
           load8<XK>(p.X, static_cast<size_t>(t) * p.K + 8 * tid, v);
         }
@@ -460,7 +504,7 @@ cudaError_t launch_t(const RowsParams &p, size_t smem, const LaunchCtx &ctx) {
     if (cudaFuncGetAttributes(&a, kern) != cudaSuccess || a.numRegs <= 0) return 16;
     const int regs = (a.numRegs + 7) / 8 * 8;  // allocation granularity
     const int w = 32768 / (32 * regs);
-    return w < 2 ? 2 : (w > kMaxWarps ? kMaxWarps : w);
+    return w < 2 ? 2 : (w > warp_cap<MT>() ? warp_cap<MT>() : w);
   }();
   const int rpc = rows_per_cta(p.N, p.ctas);
   const int want = (rpc + p.rpw - 1) / p.rpw;

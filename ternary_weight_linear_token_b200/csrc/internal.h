@@ -46,6 +46,13 @@ cudaError_t launch_decode(const void *X, int x_kind, const float *s, const uint8
                           const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                           void *Y, int y_kind, bool weights_static, const LaunchCtx &ctx);
 
+// gemv_mma.cu: int8 mma.sync with the tokens as the A operand, M <= 32,
+// K % 64 == 0; xq from launch_quantize_act(permuted = true).
+bool mmv_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_mmv(const int8_t *xq, const float *s, const uint8_t *packed, const float *gamma,
+                       int64_t M, int64_t N, int64_t K, bool relu2, void *Y, int y_kind,
+                       bool weights_static, const LaunchCtx &ctx);
+
 // gemm_generic.cu: any M, K % 16 == 0, int8 activations already quantised.
 cudaError_t launch_generic(const int8_t *xq, const float *s, const uint8_t *packed,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,

@@ -61,6 +61,10 @@ template <int KIND, bool PERM>
 __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const void *X, int64_t M,
                                                                          int64_t K, int8_t *xq,
                                                                          float *s) {
+  // Let the next kernel (the product that reads xq) launch now: its CTAs can
+  // set up and prefetch their weights while this grid runs; its own
+  // grid-dependency wait still lasts until this grid has completed.
+  pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
@@ -139,12 +143,97 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
     }
     if (lane == 0) s[m] = sm;
   }
+}
+
+// Few tokens: one CTA per row, 8 warps splitting it, so that a long row is
+// not one warp's chain of dependent loads.  Each thread keeps at most
+// kRowChunks 16-element chunks in registers (K <= 8 * 32 * 16 * kRowChunks);
+// max |x| is reduced over the warps in shared memory.
+constexpr int kRowChunks = 2;
+constexpr int kRowThreads = 256;
+constexpr int64_t kRowMaxK = int64_t(kRowThreads) * 16 * kRowChunks;
+
+template <int KIND, bool PERM>
+__global__ void __launch_bounds__(kRowThreads) quantize_row_kernel(const void *X, int64_t K,
+                                                                   int8_t *xq, float *s) {
+  __shared__ float wmax[kRowThreads / 32];
   pdl_launch_dependents();
+  pdl_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t m = blockIdx.x;
+  constexpr int kWords = KIND == kF32 ? 4 : 2;  // uint4 per 16 elements
+  const int64_t chunks = K / 16;
+  const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(X) +
+                                                    m * K * (KIND == kF32 ? 4 : 2));
+  uint4 raw[kRowChunks][kWords];
+  uint32_t amax_bits = 0;  // |x| of a float (or of a bf16) orders as an unsigned integer
+#pragma unroll
+  for (int i = 0; i < kRowChunks; ++i) {
+    const int64_t c = tid + int64_t(i) * kRowThreads;
+    if (c < chunks) {
+#pragma unroll
+      for (int j = 0; j < kWords; ++j) raw[i][j] = row[c * kWords + j];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRowChunks; ++i) {
+    if (tid + int64_t(i) * kRowThreads < chunks) {
+#pragma unroll
+      for (int j = 0; j < kWords; ++j) {
+        const uint32_t w[4] = {raw[i][j].x, raw[i][j].y, raw[i][j].z, raw[i][j].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          if (KIND == kF32) {
+            amax_bits = max(amax_bits, w[h] & 0x7FFFFFFFu);
+          } else {
+            amax_bits = max(amax_bits, (w[h] & 0x7FFFu) << 16);
+            amax_bits = max(amax_bits, w[h] & 0x7FFF0000u);
+          }
+        }
+      }
+    }
+  }
+  amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
+  if (lane == 0) wmax[warp] = __uint_as_float(amax_bits);
+  __syncthreads();
+  float amax = wmax[0];
+#pragma unroll
+  for (int i = 1; i < kRowThreads / 32; ++i) amax = fmaxf(amax, wmax[i]);
+  const float sm = act_scale(amax);
+#pragma unroll
+  for (int i = 0; i < kRowChunks; ++i) {
+    const int64_t c = tid + int64_t(i) * kRowThreads;
+    if (c < chunks) {
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < kWords; ++j) {
+        const uint32_t w[4] = {raw[i][j].x, raw[i][j].y, raw[i][j].z, raw[i][j].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          if (KIND == kF32) {
+            v[4 * j + h] = __uint_as_float(w[h]);
+          } else {
+            v[8 * j + 2 * h] = __uint_as_float(w[h] << 16);
+            v[8 * j + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+          }
+        }
+      }
+      int q[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
+      *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) =
+          PERM ? pack_permuted(q)
+               : make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                            pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
+    }
+  }
+  if (tid == 0) s[m] = sm;
 }
 
 template <int XK, int YK>
 __global__ void __launch_bounds__(32 * kRowsPerCta) rms_norm_kernel(const void *X, int64_t M,
                                                                      int64_t K, void *Y) {
+  pdl_launch_dependents();  // the next kernel may set up while this one runs
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
@@ -182,13 +271,20 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) rms_norm_kernel(const void *
       }
     }
   }
-  pdl_launch_dependents();
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
                                 float *s, bool permuted, const LaunchCtx &ctx) {
+  if (M <= ctx.num_sms && K <= kRowMaxK) {  // few tokens: one CTA per row
+    const dim3 grid(static_cast<unsigned>(M)), block(kRowThreads);
+    if (x_kind == kF32)
+      return permuted ? launch_k(quantize_row_kernel<kF32, true>, grid, block, 0, ctx, X, K, xq, s)
+                      : launch_k(quantize_row_kernel<kF32, false>, grid, block, 0, ctx, X, K, xq, s);
+    return permuted ? launch_k(quantize_row_kernel<kBF16, true>, grid, block, 0, ctx, X, K, xq, s)
+                    : launch_k(quantize_row_kernel<kBF16, false>, grid, block, 0, ctx, X, K, xq, s);
+  }
   const dim3 grid(static_cast<unsigned>(ceil_div(M, kRowsPerCta)));
   const dim3 block(32 * kRowsPerCta);
   if (x_kind == kF32)

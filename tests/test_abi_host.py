@@ -94,12 +94,15 @@ def test_matmul_rejects_bad_arguments(tw):
 
 def test_workspace_sizes(tw):
     f = tw.lib.bitnet_w158a8_matmul_workspace_size
-    assert f(1, 2560, 2560, tw.BF16) == 0          # decode, M <= 8: fused, no scratch
-    assert f(8, 6912, 2560, tw.F32) == 0
-    assert f(32, 2560, 6912, tw.BF16) == 32 * 6912 + 256   # M > 8: quantised once
+    assert f(1, 2560, 2560, tw.BF16) == 0          # decode, M <= 3: fused, no scratch
+    assert f(3, 6912, 2560, tw.F32) == 0
+    assert f(4, 6912, 2560, tw.F32) == 4 * 2560 + 256      # M >= 4: quantised once
+    assert f(8, 6912, 2560, tw.F32) == 8 * 2560 + 256
+    assert f(8, 6912, 2560, tw.I8) == 0                   # xq given
+    assert f(32, 2560, 6912, tw.BF16) == 32 * 6912 + 256
     assert f(4096, 6912, 2560, tw.I8) == 0          # xq given
     assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4
-    assert f(5, 64, 48, tw.F32) == 0                # M <= 8: fused low-latency kernel, any K
+    assert f(5, 64, 48, tw.F32) == 0                # M <= 8 and K % 64 != 0: fused kernel
     assert f(9, 64, 48, tw.F32) == 512 + 256        # generic path (M > 8, K % 64 != 0)
     assert tw.lib.bitnet_quantize_weights_workspace_size(2560, 2560) == 2560 * 8
     assert tw.lib.bitnet_quantize_weights_workspace_size(3, 16) == 256
