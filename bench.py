@@ -199,9 +199,52 @@ def make_decode(tw, torch, dev, l2_bytes):
                 "timing": "CUDA graph of the timed steps, programmatic dependent launch, "
                           "weights flagged static"},
         kernel_key="decode_gemv_M1_K2560_N2560",
-        kernel_files=["ternary_weight_linear_token_b200/csrc/gemv_decode.cu",
+        kernel_files=["ternary_weight_linear_token_b200/csrc/gemv_rows.cu",
                       "ternary_weight_linear_token_b200/csrc/common.cuh"],
         e2e_inputs=lambda: (d["x_bits"].view(np.int16), 2 * d["K"], 2 * d["N"]),
+    )
+
+
+def make_sweep(tw, torch, dev, l2_bytes, M=8):
+    """Decode sweep: one step is one decoder layer's four projections (qkv,
+    o, up + ReLU^2, down) at M tokens, each a dependent call."""
+    import synth
+    projs = []
+    for p in range(4):
+        d = synth.config_inputs("sweep", M=M, proj=p)
+        packed, gamma = tw.bitnet_quantize_weights(torch.from_numpy(d["W"]).to(dev))
+        X = torch.from_numpy(d["x_bits"].view(np.int16)).to(dev).view(torch.bfloat16)
+        Y = torch.empty((M, d["N"]), dtype=torch.bfloat16, device=dev)
+        need = tw.bitnet_w158a8_matmul_workspace_size(M, d["N"], d["K"], torch.bfloat16)
+        ws = torch.empty(max(1, need), dtype=torch.uint8, device=dev)
+        projs.append(dict(packed=packed, gamma=gamma, X=X, Y=Y, ws=ws, relu2=d["relu2"], d=d))
+    wbytes = sum(q["packed"].numel() for q in projs)
+    R = max(4, -(-3 * l2_bytes // wbytes))
+    for q in projs:  # rotating copies: every step streams its weights from HBM
+        q["copies"] = torch.empty((R,) + tuple(q["packed"].shape), dtype=torch.uint8, device=dev)
+        q["copies"][:] = q["packed"]
+
+    def step(i, stream=None):
+        for q in projs:
+            tw.bitnet_w158a8_matmul(q["X"], q["copies"][i % R], q["gamma"], relu2=q["relu2"],
+                                    Y=q["Y"], workspace=q["ws"], weights_static=True,
+                                    stream=stream)
+
+    d0 = projs[0]["d"]
+    launches = 4 if M <= 3 else 8  # 4 tokens and more: quantiser + product per projection
+    return dict(
+        step=step, kernel_step=step, units_per_step=wbytes, unit="GB/s", scale=1e-9, bound="hbm",
+        launches_per_step=launches, X=projs[0]["X"], Y=projs[3]["Y"], rotate=R,
+        config={"workload": f"decode sweep M={M}: one decoder layer's BitLinears, qkv 2560->3840, "
+                            "o 2560->2560, up 2560->6912 + ReLU^2, down 6912->2560; Student-t(3) "
+                            "bf16 activations, absmean ternary weights from N(0,0.02), bf16 out",
+                "M": M, "x_dtype": "bf16", "y_dtype": "bf16",
+                "l2": f"inputs larger than L2: {R} rotating copies of the layer's weights, "
+                      f"{R * wbytes / 1e6:.0f} MB >= 3x L2",
+                "timing": "CUDA graph of the timed steps, programmatic dependent launch, "
+                          "weights flagged static"},
+        kernel_key=None, kernel_files=[],
+        e2e_inputs=lambda: (d0["x_bits"].view(np.int16), 2 * M * d0["K"], 2 * M * 2560),
     )
 
 
@@ -284,7 +327,8 @@ def make_chain(tw, torch, dev, l2_bytes, layers=30, persistent=False):
     )
 
 
-MAKERS = {"decode": make_decode, "prefill": make_prefill, "chain": make_chain}
+MAKERS = {"decode": make_decode, "prefill": make_prefill, "chain": make_chain,
+          "sweep": make_sweep}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -308,7 +352,7 @@ def oracle_sample(workload: str, budget_s: float):
         dt = time.perf_counter() - t0
         ops = 2 * rows * n * d["N"] * d["K"]
         return ops / dt * 1e-12, "TOPS", R.num_threads(), f"{n * rows} token rows x N=6912 x K=2560", dt
-    if workload == "chain":
+    if workload in ("chain", "sweep"):
         d = synth.config_inputs("sweep", M=1, proj=2)
     else:
         d = synth.config_inputs("decode")
@@ -363,6 +407,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--sweep-m", type=int, default=8, help="sweep workload: tokens per call")
     ap.add_argument("--chain-mode", choices=["persistent", "per-launch"], default="per-launch",
                     help="chain workload: one persistent kernel per token, or one launch per step")
     args = ap.parse_args()
@@ -388,6 +433,8 @@ def main():
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2**20))
     extra = {"persistent": args.chain_mode == "persistent"} if args.workload == "chain" else {}
+    if args.workload == "sweep":
+        extra = {"M": args.sweep_m}
     w = MAKERS[args.workload](tw, torch, dev, l2, **extra)
     stream = torch.cuda.Stream(dev)
 

@@ -154,3 +154,23 @@ def test_decode_chain_matches_per_launch_chain(tw):
     Ws = [synth.layer_weights(li, p) for li in range(2) for p in range(4)]
     check_links(steps, Ws, x0["x_bits"].reshape(-1), pers.outs[-1][4].view(-1))
     assert tw.bitnet_get_device_status() == tw.OK
+
+
+def test_decode_chain_bounded_wait_reports_timeout(tw):
+    """A wait that never completes gives up (about 2 s) and is reported, with
+    no fault: the finished-CTA counter in a zero-filled workspace is set to 1,
+    so the count CTA 0 waits for at the end never appears.  The links computed
+    before that are still right, the device status is BITNET_ERR_TIMEOUT, and
+    the launch counter is not advanced (zero the workspace again after a
+    timeout, as the header says)."""
+    steps, Ws = build_chain(tw, SHAPES_A[:2], 31)
+    arr = tw.bitnet_decode_chain_steps(steps)
+    ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
+    ws.view(torch.int32)[32] = 1  # byte 128: the finished-CTA counter
+    assert tw.bitnet_get_device_status() == tw.OK
+    x0 = x0_bits(SHAPES_A[0][1], 7)
+    tw.bitnet_decode_chain(arr, bf16_t(x0), ws)
+    assert tw.bitnet_get_device_status() == tw.ERR_TIMEOUT
+    check_links(steps, Ws, x0)
+    assert int(ws.view(torch.int32)[0].item()) == 0  # launch counter unchanged
+    assert tw.bitnet_get_device_status() == tw.OK   # reading the status cleared it
