@@ -115,6 +115,9 @@ SHAPES = [
     (33, 300, 192), (128, 256, 128), (129, 257, 2624), (300, 600, 2560), (256, 520, 64),
     (384, 300, 640), (1000, 512, 2560), (640, 1100, 384),
     (5, 77, 48), (40, 33, 80), (1, 19, 2576), (130, 70, 208),
+    # 4..8 tokens quantised inside the mma.sync kernel: one K step (fewer than
+    # the warps), N below one 8-row block, an odd step count, the largest K
+    (4, 7, 64), (7, 9, 192), (4, 2000, 1088), (5, 1201, 4096), (8, 2560, 4160),
 ]
 
 
@@ -165,7 +168,7 @@ def test_matmul_degenerate(tw):
     K, N = 256, 48
     x = np.random.default_rng(5).standard_normal((3, K)).astype(np.float32)
     x[1] = 0.0  # all-zero token row -> s = 1, y row = 0
-    for path_M in (3, 40):  # decode and prefill paths
+    for path_M in (3, 6, 40):  # fused one-launch kernels and the prefill path
         xm = np.resize(x, (path_M, K)).astype(np.float32)
         Xd = f32_t(xm)
         for Wv, label in ((np.zeros((N, K), np.float32), "zero"), (np.ones((N, K), np.float32), "ones")):
