@@ -146,8 +146,12 @@ bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M
  *   flags    0 or BITNET_FLAG_WEIGHTS_STATIC.
  * Up to 3 tokens (8 when K % 64 != 0) run one fused kernel and need no
  * workspace.  Otherwise fp32/bf16 input is first quantised into the
- * workspace by the activation quantiser; then 4..32 tokens run an int8
- * mma.sync kernel and larger M the tcgen05 tensor-core kernel.
+ * workspace by the activation quantiser (M*K bytes + 4*M, each rounded up to
+ * 256); then 4..32 tokens run an int8 mma.sync kernel and larger M the
+ * tcgen05 tensor-core kernel, which first expands the packed weights to int8
+ * in the workspace (N*K more bytes, rounded up to 256; needed for int8 input
+ * too).  The weights in HBM stay packed; the int8 copy is scratch of the
+ * call.
  * ---------------------------------------------------------------------- */
 size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype);
 
@@ -198,8 +202,9 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
  * allocates nothing.
  *   - A call whose scratch need, bitnet_w158a8_matmul_workspace_size(M, N,
  *     K, x_dtype), is larger than BITNET_STATIC_SCRATCH_BYTES returns
- *     BITNET_ERR_WORKSPACE and launches nothing.  The need is 0 for int8
- *     input and for up to 3 tokens, and about M*K bytes otherwise.
+ *     BITNET_ERR_WORKSPACE and launches nothing.  The need is 0 for up to
+ *     3 tokens, about M*K bytes for 4..32 tokens, and about (M + N)*K bytes
+ *     on the tensor-core path (M*K of them only for fp32/bf16 input).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -208,7 +213,7 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
  *     whose kernels overlap on the GPU (different streams or threads) race
  *     on the array: keep them on one stream or otherwise serialised.
  * ---------------------------------------------------------------------- */
-#define BITNET_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+#define BITNET_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 
 bitnet_status bitnet_w158a8_matmul_noalloc(const void *X, bitnet_dtype x_dtype, const float *s,
                                            const uint8_t *packed, const float *gamma, int64_t M,

@@ -238,7 +238,7 @@ def bitnet_rms_norm_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: 
     return Y
 
 
-STATIC_SCRATCH_BYTES = 16 << 20
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def bitnet_w158a8_matmul_noalloc(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,

@@ -11,7 +11,8 @@
 //   decode   9 <= M <= 32, K % 64 == 0, int8 input (natural K order): the
 //            int8 mma.sync kernel with the weights as the A operand.
 //   prefill  otherwise, K % 64 == 0: bitnet_quantize_act into the workspace
-//            (unless xq is given), then the tcgen05 tensor-core kernel.
+//            (unless xq is given), the weights expanded to int8 into the
+//            workspace, then the tcgen05 tensor-core kernel.
 //   generic  K % 64 != 0: quantise into the workspace, then the dp4a kernel.
 #include <cuda_runtime.h>
 
@@ -103,14 +104,28 @@ bool use_rows(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
          (x_dtype == BITNET_I8 || M < kMmvMinM || !mmv_supported(M, N, K));
 }
 
-// Scratch the matmul needs: int8 xq [M][K] and fp32 s [M] whenever the
-// activation quantiser runs as its own kernel (every path but the fused
-// one, with float input).  Pure arithmetic: no CUDA call.
-size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
-  if (M <= 0 || N <= 0 || K <= 0 || x_dtype == BITNET_I8) return 0;
-  if (use_rows(M, N, K, x_dtype)) return 0;
+// The tensor-core path serves this call (by shape; at run time it also
+// needs the driver's tensor-map encoder, else the generic kernel runs, whose
+// scratch is a prefix of this path's).
+bool use_prefill(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
+  if (use_rows(M, N, K, x_dtype)) return false;
+  if (x_dtype == BITNET_I8 ? decode_supported(M, N, K) : mmv_supported(M, N, K)) return false;
+  return prefill_shape_ok(M, N, K);
+}
+
+// Scratch the matmul needs, in this order: int8 xq [M][K] and fp32 s [M]
+// whenever the activation quantiser runs as its own kernel (float input,
+// every path but the fused one), then the int8 weights [N][K] on the
+// tensor-core path.  Pure arithmetic: no CUDA call.
+size_t act_scratch(int64_t M, int64_t K) {
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
          align256(4 * static_cast<size_t>(M));
+}
+size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (use_rows(M, N, K, x_dtype)) return 0;
+  const size_t act = x_dtype == BITNET_I8 ? 0 : act_scratch(M, K);
+  return act + (use_prefill(M, N, K, x_dtype) ? align256(prefill_weight_bytes(N, K)) : 0);
 }
 
 // Argument checks of bitnet_w158a8_matmul (and of its normalising variant,
@@ -161,7 +176,7 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
   const bool from_float = x_dtype != BITNET_I8;
   const bool mmv = from_float && mmv_supported(M, N, K);
   const bool decode = !from_float && decode_supported(M, N, K);  // caller's int8, 9..32 tokens
-  const bool prefill = !mmv && !decode && prefill_supported(M, N, K);
+  const bool prefill = use_prefill(M, N, K, x_dtype) && prefill_supported(M, N, K);
   const int8_t *xq = static_cast<const int8_t *>(X);
   const float *sq = s;
   if (from_float) {
@@ -182,7 +197,9 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                                    wstatic, ctx));
   if (prefill)
     return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                    from_float, ctx));
+                                    from_float,
+                                    static_cast<int8_t *>(workspace) + (from_float ? act_scratch(M, K) : 0),
+                                    ctx));
   return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
 }
 

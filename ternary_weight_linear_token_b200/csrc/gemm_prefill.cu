@@ -4,28 +4,32 @@
 // the ternary weights {-1, 0, +1} held as int8 (BitNet b1.58 2B4T model card,
 // 模型详情 -> 量化: W1.58A8; "Microsoft BitNet 深度研究报告", 技术原理 items 2-3).
 //
-// Persistent kernel, one CTA per SM, output tiles of 128 tokens x 256
-// features taken round-robin; K in 128-byte stages.
-//   warp 4      TMA producer: xq tile [128 x 128 B] (128-byte swizzle) and the
-//               packed weight tile [256 rows x 32 B] -- 2 bits per weight all
-//               the way from HBM into shared memory -- into a 5-stage ring.
-//   warps 6-21  expand each packed word into 16 int8 weights, stored as the
-//               K-major 128-byte-swizzled B operand in a 2-stage ring.
-//   warp 5      allocates 512 TMEM columns (two 256-column accumulators); one
+// Two kernels per call:
+//   expand_weights_kernel  the packed 2-bit weights -> int8 [N][K] in a
+//               workspace (one coalesced pass: 4.4 MB in, 17.7 MB out for
+//               6912 x 2560), in the K order of the activations: permuted
+//               inside each 16-element group (four byte-permute lookups per
+//               word) for activations quantised by this library, natural
+//               (shift/mask/multiply) for int8 activations given by the caller.
+//   prefill_kernel  persistent, one CTA per SM, output tiles of 128 tokens x
+//               256 features taken round-robin; K in 128-byte stages.
+//     warp 4    TMA producer: the xq tile [128 x 128 B] and the int8 weight
+//               tile [256 x 128 B], both 128-byte swizzled, into a 4-stage ring.
+//     warp 5    allocates 512 TMEM columns (two 256-column accumulators); one
 //               lane issues 4 MMAs (M=128, N=256, K=32) per stage and commits
-//               them to the barriers that free the TMA and B stages, and,
-//               after a tile's last stage, to the accumulator-full barrier.
-//   warps 0-3   epilogue: tcgen05.ld of the finished accumulator, y = acc *
+//               them to the barrier that frees the stage, and, after a tile's
+//               last stage, to the accumulator-full barrier.
+//     warps 0-3 epilogue: tcgen05.ld of the finished accumulator, y = acc *
 //               (gamma / s_m), optional ReLU^2; bf16 output goes through a
 //               128-byte-swizzled shared-memory staging block (32 rows x 64
 //               columns per warp, double-buffered) and a TMA tensor store,
 //               so HBM sees whole lines; then the accumulator is released,
 //               so tile i's epilogue overlaps tile i+1's MMAs.
-// Expansion: with activations quantised by this library (int8 in a K order
-// permuted inside each 16-element group) a packed word becomes 16 weights by
-// four byte-permute lookups (3 instructions per 4 weights); with int8
-// activations given by the caller (natural K order) it uses the in-order
-// shift/mask/multiply unpack.  Every wait is bounded (see common.cuh).
+// Expanding in HBM first keeps shared memory for the tensor core's operands
+// only: per 128-byte K stage it carries the TMA writes (48 KB) and the
+// operand reads (48 KB); expanding inside the kernel added the packed reads
+// and the expanded stores (40 KB more) and bounded the kernel by shared-memory
+// bandwidth.  Every wait is bounded (see common.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -38,25 +42,23 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int kTmaStages = 5;
-constexpr int kBxStages = 2;
+constexpr int kStages = 4;
 constexpr int kEpiWarps = 4;
-constexpr int kExpWarps = 16;
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
-constexpr int kWarpExp0 = 6;
-constexpr int kThreads = 32 * (kEpiWarps + 2 + kExpWarps);
+constexpr int kThreads = 32 * (kEpiWarps + 2);
 constexpr int kABytes = BM * BK;
-constexpr int kBpBytes = BN * BK / 4;
-constexpr int kTmaStageBytes = kABytes + kBpBytes;
-constexpr int kBxBytes = BN * BK;
+constexpr int kBBytes = BN * BK;
+constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * BN;
-constexpr int kStageRows = 32;                    // epilogue staging block: 32 rows
-constexpr int kStageCols = 64;                    // x 64 bf16 columns = 128-byte rows
-constexpr int kStageBytes = kStageRows * kStageCols * 2;
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kTmaStages) * kTmaStageBytes +
-                              kBxStages * kBxBytes + kEpiWarps * 2 * kStageBytes + 256;
+constexpr int kStoreRows = 32;                    // epilogue staging block: 32 rows
+constexpr int kStoreCols = 64;                    // x 64 bf16 columns = 128-byte rows
+constexpr int kStoreBytes = kStoreRows * kStoreCols * 2;
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes +
+                              kEpiWarps * 2 * kStoreBytes + 256;
 constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
+constexpr int kExpandThreads = 256;
+constexpr int kExpandWords = 4;                   // packed words per thread
 
 // Instruction descriptor: s8 x s8 -> s32, both operands K-major, M=128, N=256.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) |
@@ -137,7 +139,32 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
                     unpack_natural(w, 3));
 }
 
-template <int YK, bool RELU2, bool PERM, bool TMA_Y>
+// Packed word w (16 weights) -> bytes 16w..16w+15 of the int8 weights: the
+// packed matrix [N][K/16 words] and the int8 one [N][K] share their row
+// order, so the flat word index maps straight through.  A warp handles 128
+// consecutive words per pass: 4-byte loads and 16-byte stores, both
+// contiguous across the warp.
+template <bool PERM>
+__global__ void __launch_bounds__(kExpandThreads)
+    expand_weights_kernel(const uint32_t *packed, uint4 *w8, int64_t words) {
+  pdl_launch_dependents();
+  pdl_wait();  // the previous product may still be reading this buffer
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * (kExpandThreads * kExpandWords) +
+                       (threadIdx.x >> 5) * (32 * kExpandWords) + (threadIdx.x & 31);
+  uint32_t w[kExpandWords];
+#pragma unroll
+  for (int j = 0; j < kExpandWords; ++j) {
+    const int64_t i = base + 32 * j;
+    w[j] = i < words ? packed[i] : 0u;
+  }
+#pragma unroll
+  for (int j = 0; j < kExpandWords; ++j) {
+    const int64_t i = base + 32 * j;
+    if (i < words) w8[i] = expand_word<PERM>(w[j]);
+  }
+}
+
+template <int YK, bool RELU2, bool TMA_Y>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
@@ -145,14 +172,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *tma_ring = smem;
-  uint8_t *bx_ring = smem + kTmaStages * kTmaStageBytes;
-  uint8_t *staging = bx_ring + kBxStages * kBxBytes;   // [kEpiWarps][2][32 x 128 B]
-  uint64_t *tma_full = reinterpret_cast<uint64_t *>(staging + kEpiWarps * 2 * kStageBytes);
-  uint64_t *tma_empty = tma_full + kTmaStages;
-  uint64_t *bx_full = tma_empty + kTmaStages;
-  uint64_t *bx_empty = bx_full + kBxStages;
-  uint64_t *acc_full = bx_empty + kBxStages;
+  uint8_t *ring = smem;                                 // [kStages][A 16 KB | B 32 KB]
+  uint8_t *staging = ring + kStages * kStageBytes;      // [kEpiWarps][2][32 x 128 B]
+  uint64_t *full = reinterpret_cast<uint64_t *>(staging + kEpiWarps * 2 * kStoreBytes);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;
   uint64_t *acc_empty = acc_full + 2;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
@@ -161,13 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = p.m_tiles * p.n_tiles;
 
   if (warp == kWarpTma && lane == 0) {
-    for (int s = 0; s < kTmaStages; ++s) {
-      mbar_init(&tma_full[s], 1);
-      mbar_init(&tma_empty[s], 1);
-    }
-    for (int b = 0; b < kBxStages; ++b) {
-      mbar_init(&bx_full[b], kExpWarps);
-      mbar_init(&bx_empty[b], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
@@ -198,15 +218,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int32_t m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kTmaStages;
-          if (it >= kTmaStages && !mbar_wait(&tma_empty[s], ((it / kTmaStages) - 1) & 1, p.status)) {
+          const int s = it % kStages;
+          if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, p.status)) {
             ok = false;
             break;
           }
-          uint8_t *stage = tma_ring + s * kTmaStageBytes;
-          mbar_arrive_expect_tx(&tma_full[s], kTmaStageBytes);
-          tma_load_2d(stage, &tmap_a, kb * BK, m0, &tma_full[s]);
-          tma_load_2d(stage + kABytes, &tmap_b, kb * (BK / 4), n0, &tma_full[s]);
+          uint8_t *stage = ring + s * kStageBytes;
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          tma_load_2d(stage, &tmap_a, kb * BK, m0, &full[s]);
+          tma_load_2d(stage + kABytes, &tmap_b, kb * BK, n0, &full[s]);
         }
       }
     }
@@ -221,54 +241,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kTmaStages, b = it % kBxStages;
-          ok = mbar_wait(&tma_full[s], (it / kTmaStages) & 1, p.status) &&
-               mbar_wait(&bx_full[b], (it / kBxStages) & 1, p.status);
+          const int s = it % kStages;
+          ok = mbar_wait(&full[s], (it / kStages) & 1, p.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(tma_ring + s * kTmaStageBytes);
-          const uint32_t b_base = smem_u32(bx_ring + b * kBxBytes);
+          const uint32_t a_base = smem_u32(ring + s * kStageBytes);
+          const uint32_t b_base = a_base + kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
             mma_i8(d, smem_desc_sw128(a_base + 32 * kk), smem_desc_sw128(b_base + 32 * kk), kIdesc,
                    (kb | kk) != 0 ? 1u : 0u);
-          mma_commit(&tma_empty[s]);
-          mma_commit(&bx_empty[b]);
+          mma_commit(&empty[s]);
         }
         mma_commit(&acc_full[acc]);
-      }
-    }
-  } else if (warp >= kWarpExp0) {
-    // ---- expansion: packed [256 rows x 32 B] -> int8 [256 x 128] K-major SW128
-    const int et = (warp - kWarpExp0) * 32 + lane;
-    uint32_t it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < kblocks; ++kb, ++it) {
-        const int s = it % kTmaStages, b = it % kBxStages;
-        if (!mbar_wait(&tma_full[s], (it / kTmaStages) & 1, p.status) ||
-            (it >= kBxStages && !mbar_wait(&bx_empty[b], ((it / kBxStages) - 1) & 1, p.status))) {
-          ok = false;
-          break;
-        }
-        const uint8_t *bp = tma_ring + s * kTmaStageBytes + kABytes;
-        uint8_t *bx = bx_ring + b * kBxBytes;
-        uint32_t w[(BN * BK / 16) / (32 * kExpWarps)];
-#pragma unroll
-        for (int i = 0; i < (BN * BK / 16) / (32 * kExpWarps); ++i) {
-          const int wi = et + 32 * kExpWarps * i;
-          w[i] = *reinterpret_cast<const uint32_t *>(bp + (wi >> 3) * 32 + (wi & 7) * 4);
-        }
-#pragma unroll
-        for (int i = 0; i < (BN * BK / 16) / (32 * kExpWarps); ++i) {
-          const int wi = et + 32 * kExpWarps * i;
-          const int r = wi >> 3, c = wi & 7;
-          *reinterpret_cast<uint4 *>(bx + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
-              expand_word<PERM>(w[i]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bx_full[b]);
       }
     }
   } else {
@@ -276,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp;
     const float gamma = *p.gamma;
     const bool vec_ok = (YK == kBF16) ? (p.N % 8 == 0) : (p.N % 4 == 0);
-    uint8_t *my_stage = staging + q * 2 * kStageBytes;
+    uint8_t *my_stage = staging + q * 2 * kStoreBytes;
     int tl = 0, stores = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tl) {
       const int acc = tl & 1;
@@ -290,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (static_cast<uint32_t>(q * 32) << 16);
       if (TMA_Y) {
 #pragma unroll 1
-        for (int cb = 0; cb < BN / kStageCols; ++cb, ++stores) {
-          uint8_t *buf = my_stage + (stores & 1) * kStageBytes;
+        for (int cb = 0; cb < BN / kStoreCols; ++cb, ++stores) {
+          uint8_t *buf = my_stage + (stores & 1) * kStoreBytes;
           if (stores >= 2) {  // the store that last used this buffer has read it
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
@@ -299,12 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t v[32];
-            tmem_ld16(t_row + static_cast<uint32_t>(cb * kStageCols + 32 * half),
+            tmem_ld16(t_row + static_cast<uint32_t>(cb * kStoreCols + 32 * half),
                       *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-            tmem_ld16(t_row + static_cast<uint32_t>(cb * kStageCols + 32 * half + 16),
+            tmem_ld16(t_row + static_cast<uint32_t>(cb * kStoreCols + 32 * half + 16),
                       *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
             tmem_wait_ld();
-            if (cb == BN / kStageCols - 1 && half == 1) {  // accumulator fully read
+            if (cb == BN / kStoreCols - 1 && half == 1) {  // accumulator fully read
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -327,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmap_y, buf, static_cast<int32_t>(n0 + cb * kStageCols),
+            tma_store_2d(&tmap_y, buf, static_cast<int32_t>(n0 + cb * kStoreCols),
                          static_cast<int32_t>(m_base));
             bulk_commit();
           }
@@ -380,10 +365,10 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YK, bool RELU2, bool PERM, bool TMA_Y>
+template <int YK, bool RELU2, bool TMA_Y>
 cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
                const PrefillParams &p, const LaunchCtx &ctx) {
-  auto kern = prefill_kernel<YK, RELU2, PERM, TMA_Y>;
+  auto kern = prefill_kernel<YK, RELU2, TMA_Y>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
@@ -392,36 +377,47 @@ cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &
   return launch_k(kern, grid, dim3(kThreads), kSmemBytes, ctx, ta, tb, ty, p);
 }
 
-template <bool PERM>
 cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, bool tma_y,
                  const PrefillParams &p, int y_kind, bool relu2, const LaunchCtx &ctx) {
-  if (y_kind == kI32) return go<kI32, false, PERM, false>(ta, tb, ty, p, ctx);
+  if (y_kind == kI32) return go<kI32, false, false>(ta, tb, ty, p, ctx);
   if (y_kind == kF32)
-    return relu2 ? go<kF32, true, PERM, false>(ta, tb, ty, p, ctx)
-                 : go<kF32, false, PERM, false>(ta, tb, ty, p, ctx);
+    return relu2 ? go<kF32, true, false>(ta, tb, ty, p, ctx) : go<kF32, false, false>(ta, tb, ty, p, ctx);
   if (tma_y)
-    return relu2 ? go<kBF16, true, PERM, true>(ta, tb, ty, p, ctx)
-                 : go<kBF16, false, PERM, true>(ta, tb, ty, p, ctx);
-  return relu2 ? go<kBF16, true, PERM, false>(ta, tb, ty, p, ctx)
-               : go<kBF16, false, PERM, false>(ta, tb, ty, p, ctx);
+    return relu2 ? go<kBF16, true, true>(ta, tb, ty, p, ctx) : go<kBF16, false, true>(ta, tb, ty, p, ctx);
+  return relu2 ? go<kBF16, true, false>(ta, tb, ty, p, ctx) : go<kBF16, false, false>(ta, tb, ty, p, ctx);
 }
 
 }  // namespace
 
-bool prefill_supported(int64_t M, int64_t N, int64_t K) {
-  return M >= 1 && N >= 1 && K % 64 == 0 && ceil_div(M, BM) * ceil_div(N, BN) < (1LL << 31) &&
-         encode_fn() != nullptr;
+bool prefill_shape_ok(int64_t M, int64_t N, int64_t K) {
+  return M >= 1 && N >= 1 && K % 64 == 0 && ceil_div(M, BM) * ceil_div(N, BN) < (1LL << 31);
 }
+
+bool prefill_supported(int64_t M, int64_t N, int64_t K) {
+  return prefill_shape_ok(M, N, K) && encode_fn() != nullptr;
+}
+
+size_t prefill_weight_bytes(int64_t N, int64_t K) { return static_cast<size_t>(N) * K; }
 
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, bool xq_permuted, const LaunchCtx &ctx) {
+                           void *Y, int y_kind, bool xq_permuted, int8_t *w8,
+                           const LaunchCtx &ctx) {
   CUtensorMap ta, tb;
   if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                    static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N),
-                   static_cast<uint64_t>(K / 4), BK / 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+      !make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                   static_cast<uint64_t>(K), BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  // the int8 weights, in the activations' K order
+  const int64_t words = N * (K / 16);
+  const dim3 eg(static_cast<unsigned>(ceil_div(words, int64_t{kExpandThreads} * kExpandWords)));
+  const uint32_t *pw = reinterpret_cast<const uint32_t *>(packed);
+  uint4 *w8v = reinterpret_cast<uint4 *>(w8);
+  cudaError_t e = xq_permuted
+                      ? launch_k(expand_weights_kernel<true>, eg, dim3(kExpandThreads), 0, ctx, pw, w8v, words)
+                      : launch_k(expand_weights_kernel<false>, eg, dim3(kExpandThreads), 0, ctx, pw, w8v, words);
+  if (e != cudaSuccess) return e;
   PrefillParams p;
   p.s = s;
   p.gamma = gamma;
@@ -436,11 +432,10 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *pack
   CUtensorMap ty;
   const bool tma_y = y_kind == kBF16 && N % 8 == 0 &&
                      make_map_2d(&ty, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
-                                 static_cast<uint64_t>(N) * 2, kStageCols, kStageRows,
+                                 static_cast<uint64_t>(N) * 2, kStoreCols, kStoreRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   if (!tma_y) ty = ta;  // unused by the direct-store kernels
-  return xq_permuted ? go_y<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx)
-                     : go_y<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+  return go_y(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet

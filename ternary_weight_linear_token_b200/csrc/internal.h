@@ -58,12 +58,18 @@ cudaError_t launch_generic(const int8_t *xq, const float *s, const uint8_t *pack
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                            void *Y, int y_kind, const LaunchCtx &ctx);
 
-// gemm_prefill.cu: tcgen05 tensor-core kernel, K % 64 == 0.  xq_permuted:
-// xq comes from launch_quantize_act(permuted = true).
+// gemm_prefill.cu: the weights expanded to int8 into w8 (N * K bytes of
+// scratch), then the tcgen05 tensor-core kernel; K % 64 == 0.  xq_permuted:
+// xq comes from launch_quantize_act(permuted = true).  prefill_shape_ok is
+// the shape rule alone (no CUDA call); prefill_supported also needs the
+// driver's tensor-map encoder.
+bool prefill_shape_ok(int64_t M, int64_t N, int64_t K);
 bool prefill_supported(int64_t M, int64_t N, int64_t K);
+size_t prefill_weight_bytes(int64_t N, int64_t K);
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, bool xq_permuted, const LaunchCtx &ctx);
+                           void *Y, int y_kind, bool xq_permuted, int8_t *w8,
+                           const LaunchCtx &ctx);
 
 // chain.cu: persistent M = 1 chain of BitLinear projections (one
 // cooperative launch).  Step flags mirror BITNET_STEP_*.

@@ -100,8 +100,12 @@ def test_workspace_sizes(tw):
     assert f(8, 6912, 2560, tw.F32) == 8 * 2560 + 256
     assert f(8, 6912, 2560, tw.I8) == 0                   # xq given
     assert f(32, 2560, 6912, tw.BF16) == 32 * 6912 + 256
-    assert f(4096, 6912, 2560, tw.I8) == 0          # xq given
-    assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4
+    assert f(16, 2560, 6912, tw.I8) == 0            # xq given, mma.sync path
+    # tensor-core path: xq and s (float input only), then the int8 weights
+    assert f(4096, 6912, 2560, tw.I8) == 6912 * 2560
+    assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4 + 6912 * 2560
+    assert f(33, 7, 64, tw.F32) == 2304 + 256 + 512       # each part rounded up to 256
+    assert f(40, 33, 80, tw.I8) == 0                # K % 64 != 0: generic kernel
     assert f(5, 64, 48, tw.F32) == 0                # M <= 8 and K % 64 != 0: fused kernel
     assert f(9, 64, 48, tw.F32) == 512 + 256        # generic path (M > 8, K % 64 != 0)
     assert tw.lib.bitnet_quantize_weights_workspace_size(2560, 2560) == 2560 * 8

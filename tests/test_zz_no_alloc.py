@@ -89,7 +89,7 @@ def test_noalloc_binding_and_size_limit(tw):
     y = tw.bitnet_w158a8_matmul_noalloc(X, packed, gamma)
     assert torch.equal(y, tw.bitnet_w158a8_matmul(X, packed, gamma))
     # the scratch need of this call (M*K bytes of int8 + scales) is above the
-    # built-in 16 MiB: rejected with the workspace status, nothing launched
+    # built-in scratch: rejected with the workspace status, nothing launched
     M_big = (tw.STATIC_SCRATCH_BYTES // K) + 64
     need = tw.bitnet_w158a8_matmul_workspace_size(M_big, 64, K, torch.bfloat16)
     assert need > tw.STATIC_SCRATCH_BYTES
