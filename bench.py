@@ -288,7 +288,8 @@ def make_prefill(tw, torch, dev, l2_bytes):
                             "accumulation, bf16 out",
                 "M": M, "K": K, "N": N, "x_dtype": "bf16", "y_dtype": "bf16",
                 "l2": f"inputs larger than L2: {R} rotating input/output sets",
-                "timing": "CUDA graph; step = activation quantiser + tcgen05 kernel"},
+                "timing": "CUDA graph; step = activation quantiser (the weights' expansion to "
+                          "int8 scratch runs in the same launch) + tcgen05 kernel"},
         kernel_key="prefill_tcgen05_M4096_K2560_N6912",
         kernel_files=["ternary_weight_linear_token_b200/csrc/gemm_prefill.cu",
                       "ternary_weight_linear_token_b200/csrc/common.cuh"],
@@ -545,8 +546,10 @@ def main():
             "roofline": {"bound": w["bound"], "achieved": achieved, "peak": peak, "unit": punit,
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
                          "kernel_us": 1e3 * kms / args.steps,
-                         "kernel_timing": ("step time minus the activation quantiser's time, both "
-                                           "CUDA-event timed on the launch stream")
+                         "kernel_timing": ("step time minus the time of the activation quantiser "
+                                           "alone (without the weight expansion, which the "
+                                           "kernel's figure therefore carries), both CUDA-event "
+                                           "timed on the launch stream")
                          if quant_ms is not None else "CUDA-event time of the timed steps"},
             "cpu_baseline": cpu,
             "clocks": clocks.summary(),

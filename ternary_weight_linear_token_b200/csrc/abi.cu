@@ -179,16 +179,26 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
   const bool prefill = use_prefill(M, N, K, x_dtype) && prefill_supported(M, N, K);
   const int8_t *xq = static_cast<const int8_t *>(X);
   const float *sq = s;
+  ExpandJob expand;  // the tensor-core path's int8 weights, after the activation scratch
+  if (prefill) {
+    expand.packed = packed;
+    expand.w8 = static_cast<int8_t *>(workspace) + (from_float ? act_scratch(M, K) : 0);
+    expand.words = N * (K / 16);
+  }
   if (from_float) {
     // The prefill and mmv kernels take the quantiser's output in the K order
     // of their fast weight unpack; the generic kernel wants natural order.
+    // The weight expansion rides in the quantiser's launch.
     int8_t *wxq = static_cast<int8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                           align256(static_cast<size_t>(M) * K));
-    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill || mmv, ctx);
+    cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill || mmv, ctx, expand);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     xq = wxq;
     sq = ws;
+  } else if (prefill) {
+    // the caller's int8 activations are in natural K order
+    if (launch_expand_weights(expand, false, ctx) != cudaSuccess) return BITNET_ERR_CUDA;
   }
   if (mmv)
     return from_cuda(launch_mmv(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, wstatic, ctx));
@@ -196,10 +206,7 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
     return from_cuda(launch_decode(xq, BITNET_I8, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                    wstatic, ctx));
   if (prefill)
-    return from_cuda(launch_prefill(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                                    from_float,
-                                    static_cast<int8_t *>(workspace) + (from_float ? act_scratch(M, K) : 0),
-                                    ctx));
+    return from_cuda(launch_prefill(xq, sq, expand.w8, gamma, M, N, K, relu2, Y, y_dtype, ctx));
   return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
 }
 

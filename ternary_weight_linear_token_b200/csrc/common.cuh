@@ -258,4 +258,19 @@ __device__ __forceinline__ uint4 pack_permuted(const int (&q)[16]) {
   return o;
 }
 
+// 16 int8 weights {0, +1, -1} of one packed word.  PERM: in the K order of
+// pack_permuted, by four byte-permute lookups in a 4-entry table held in a
+// register (code 0 -> 0x00, 1 -> 0x01, 2 and 3 -> 0xFF), 3 instructions per 4
+// weights; else natural order (shift/mask/multiply).
+template <bool PERM>
+__device__ __forceinline__ uint4 expand_word(uint32_t w) {
+  constexpr uint32_t kLut = 0xFFFF0100u;
+  if (PERM)
+    return make_uint4(__byte_perm(kLut, 0u, w & 0x3333u), __byte_perm(kLut, 0u, (w >> 2) & 0x3333u),
+                      __byte_perm(kLut, 0u, (w >> 16) & 0x3333u),
+                      __byte_perm(kLut, 0u, (w >> 18) & 0x3333u));
+  return make_uint4(unpack_natural(w, 0), unpack_natural(w, 1), unpack_natural(w, 2),
+                    unpack_natural(w, 3));
+}
+
 }  // namespace bitnet

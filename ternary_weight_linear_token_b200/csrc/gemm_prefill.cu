@@ -4,14 +4,10 @@
 // the ternary weights {-1, 0, +1} held as int8 (BitNet b1.58 2B4T model card,
 // 模型详情 -> 量化: W1.58A8; "Microsoft BitNet 深度研究报告", 技术原理 items 2-3).
 //
-// Two kernels per call:
-//   expand_weights_kernel  the packed 2-bit weights -> int8 [N][K] in a
-//               workspace (one coalesced pass: 4.4 MB in, 17.7 MB out for
-//               6912 x 2560), in the K order of the activations: permuted
-//               inside each 16-element group (four byte-permute lookups per
-//               word) for activations quantised by this library, natural
-//               (shift/mask/multiply) for int8 activations given by the caller.
-//   prefill_kernel  persistent, one CTA per SM, output tiles of 128 tokens x
+// The int8 weights come from the packed ones by a coalesced expansion pass
+// beforehand (launched with the activation quantiser: 4.4 MB in, 17.7 MB out
+// for 6912 x 2560), in the K order of the activations.
+// prefill_kernel: persistent, one CTA per SM, output tiles of 128 tokens x
 //               256 features taken round-robin; K in 128-byte stages.
 //     warp 4    TMA producer: the xq tile [128 x 128 B] and the int8 weight
 //               tile [256 x 128 B], both 128-byte swizzled, into a 4-stage ring.
@@ -56,9 +52,6 @@ constexpr int kStoreCols = 64;                    // x 64 bf16 columns = 128-byt
 constexpr int kStoreBytes = kStoreRows * kStoreCols * 2;
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes +
                               kEpiWarps * 2 * kStoreBytes + 256;
-constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
-constexpr int kExpandThreads = 256;
-constexpr int kExpandWords = 4;                   // packed words per thread
 
 // Instruction descriptor: s8 x s8 -> s32, both operands K-major, M=128, N=256.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) |
@@ -124,43 +117,6 @@ __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64
           reinterpret_cast<uint16_t *>(dst)[e] = static_cast<uint16_t>(bits);
         }
     }
-  }
-}
-
-// 16 int8 weights of one packed word, in the K order the A operand uses.
-template <bool PERM>
-__device__ __forceinline__ uint4 expand_word(uint32_t w) {
-  if (PERM)
-    return make_uint4(__byte_perm(kTernaryLut, 0u, w & 0x3333u),
-                      __byte_perm(kTernaryLut, 0u, (w >> 2) & 0x3333u),
-                      __byte_perm(kTernaryLut, 0u, (w >> 16) & 0x3333u),
-                      __byte_perm(kTernaryLut, 0u, (w >> 18) & 0x3333u));
-  return make_uint4(unpack_natural(w, 0), unpack_natural(w, 1), unpack_natural(w, 2),
-                    unpack_natural(w, 3));
-}
-
-// Packed word w (16 weights) -> bytes 16w..16w+15 of the int8 weights: the
-// packed matrix [N][K/16 words] and the int8 one [N][K] share their row
-// order, so the flat word index maps straight through.  A warp handles 128
-// consecutive words per pass: 4-byte loads and 16-byte stores, both
-// contiguous across the warp.
-template <bool PERM>
-__global__ void __launch_bounds__(kExpandThreads)
-    expand_weights_kernel(const uint32_t *packed, uint4 *w8, int64_t words) {
-  pdl_launch_dependents();
-  pdl_wait();  // the previous product may still be reading this buffer
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * (kExpandThreads * kExpandWords) +
-                       (threadIdx.x >> 5) * (32 * kExpandWords) + (threadIdx.x & 31);
-  uint32_t w[kExpandWords];
-#pragma unroll
-  for (int j = 0; j < kExpandWords; ++j) {
-    const int64_t i = base + 32 * j;
-    w[j] = i < words ? packed[i] : 0u;
-  }
-#pragma unroll
-  for (int j = 0; j < kExpandWords; ++j) {
-    const int64_t i = base + 32 * j;
-    if (i < words) w8[i] = expand_word<PERM>(w[j]);
   }
 }
 
@@ -399,25 +355,15 @@ bool prefill_supported(int64_t M, int64_t N, int64_t K) {
 
 size_t prefill_weight_bytes(int64_t N, int64_t K) { return static_cast<size_t>(N) * K; }
 
-cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
+cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, bool xq_permuted, int8_t *w8,
-                           const LaunchCtx &ctx) {
+                           void *Y, int y_kind, const LaunchCtx &ctx) {
   CUtensorMap ta, tb;
   if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                    static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                    static_cast<uint64_t>(K), BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // the int8 weights, in the activations' K order
-  const int64_t words = N * (K / 16);
-  const dim3 eg(static_cast<unsigned>(ceil_div(words, int64_t{kExpandThreads} * kExpandWords)));
-  const uint32_t *pw = reinterpret_cast<const uint32_t *>(packed);
-  uint4 *w8v = reinterpret_cast<uint4 *>(w8);
-  cudaError_t e = xq_permuted
-                      ? launch_k(expand_weights_kernel<true>, eg, dim3(kExpandThreads), 0, ctx, pw, w8v, words)
-                      : launch_k(expand_weights_kernel<false>, eg, dim3(kExpandThreads), 0, ctx, pw, w8v, words);
-  if (e != cudaSuccess) return e;
   PrefillParams p;
   p.s = s;
   p.gamma = gamma;

@@ -26,8 +26,18 @@ cudaError_t launch_quantize_weights(const void *W, int w_kind, int64_t N, int64_
 // quant_act.cu
 // permuted: store each 16-element group of xq in the order the byte-permute
 // weight unpack produces (internal layout of the prefill kernel's A operand).
+// The packed weights [N][K/4] expanded to int8 [N][K] (scratch of the
+// tensor-core path): words = N * K / 16 packed words, 0 for none.
+struct ExpandJob {
+  const uint8_t *packed = nullptr;
+  int8_t *w8 = nullptr;
+  int64_t words = 0;
+};
 cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
-                                float *s, bool permuted, const LaunchCtx &ctx);
+                                float *s, bool permuted, const LaunchCtx &ctx,
+                                const ExpandJob &expand = ExpandJob{});
+// The expansion alone (int8 activations given by the caller).
+cudaError_t launch_expand_weights(const ExpandJob &job, bool permuted, const LaunchCtx &ctx);
 cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
                             const LaunchCtx &ctx);
 
@@ -58,18 +68,16 @@ cudaError_t launch_generic(const int8_t *xq, const float *s, const uint8_t *pack
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                            void *Y, int y_kind, const LaunchCtx &ctx);
 
-// gemm_prefill.cu: the weights expanded to int8 into w8 (N * K bytes of
-// scratch), then the tcgen05 tensor-core kernel; K % 64 == 0.  xq_permuted:
-// xq comes from launch_quantize_act(permuted = true).  prefill_shape_ok is
-// the shape rule alone (no CUDA call); prefill_supported also needs the
-// driver's tensor-map encoder.
+// gemm_prefill.cu: the tcgen05 tensor-core kernel on int8 xq and int8
+// weights w8 [N][K] (expanded beforehand, in xq's K order); K % 64 == 0.
+// prefill_shape_ok is the shape rule alone (no CUDA call);
+// prefill_supported also needs the driver's tensor-map encoder.
 bool prefill_shape_ok(int64_t M, int64_t N, int64_t K);
 bool prefill_supported(int64_t M, int64_t N, int64_t K);
 size_t prefill_weight_bytes(int64_t N, int64_t K);
-cudaError_t launch_prefill(const int8_t *xq, const float *s, const uint8_t *packed,
+cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, bool xq_permuted, int8_t *w8,
-                           const LaunchCtx &ctx);
+                           void *Y, int y_kind, const LaunchCtx &ctx);
 
 // chain.cu: persistent M = 1 chain of BitLinear projections (one
 // cooperative launch).  Step flags mirror BITNET_STEP_*.

@@ -10,6 +10,12 @@
 // 16-byte int8 output chunk) per lane-step, four steps per lane in flight at
 // a time (a K = 2560 row is two dependent rounds of loads, not five);
 // K % 16 == 0.
+//
+// On the tensor-core path the same launch also expands the packed weights
+// into int8 scratch: blocks past the quantiser's take 1024 packed words each.
+// The quantiser is bound by its FMA/ALU issue, so the expansion's memory
+// traffic (4.4 MB in, 17.7 MB out for 6912 x 2560) runs beside it instead of
+// as a launch of its own.
 #include "common.cuh"
 #include "internal.h"
 
@@ -57,15 +63,56 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+constexpr int kExpandWords = 4;  // packed words per thread
+constexpr int64_t kExpandBlockWords = 32 * kRowsPerCta * kExpandWords;
+
+// Packed word w (16 weights) -> bytes 16w..16w+15 of the int8 weights: the
+// packed matrix [N][K/16 words] and the int8 one [N][K] share their row
+// order, so the flat word index maps straight through.  A warp handles 128
+// consecutive words: 4-byte loads and 16-byte stores, contiguous across it.
+template <bool PERM>
+__device__ __forceinline__ void expand_block(const ExpandJob &job, int64_t block) {
+  const uint32_t *packed = reinterpret_cast<const uint32_t *>(job.packed);
+  uint4 *w8 = reinterpret_cast<uint4 *>(job.w8);
+  const int64_t base = block * kExpandBlockWords + (threadIdx.x >> 5) * (32 * kExpandWords) +
+                       (threadIdx.x & 31);
+  uint32_t w[kExpandWords];
+#pragma unroll
+  for (int j = 0; j < kExpandWords; ++j) {
+    const int64_t i = base + 32 * j;
+    w[j] = i < job.words ? packed[i] : 0u;
+  }
+#pragma unroll
+  for (int j = 0; j < kExpandWords; ++j) {
+    const int64_t i = base + 32 * j;
+    if (i < job.words) w8[i] = expand_word<PERM>(w[j]);
+  }
+}
+
+template <bool PERM>
+__global__ void __launch_bounds__(32 * kRowsPerCta) expand_weights_kernel(const ExpandJob job) {
+  pdl_launch_dependents();
+  pdl_wait();  // the previous product may still be reading the scratch
+  expand_block<PERM>(job, blockIdx.x);
+}
+
+// Blocks [0, qblocks) quantise 8 token rows each; later blocks expand the
+// weights of `job` (none when job.words == 0).
 template <int KIND, bool PERM>
 __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const void *X, int64_t M,
                                                                          int64_t K, int8_t *xq,
-                                                                         float *s) {
+                                                                         float *s,
+                                                                         const ExpandJob job,
+                                                                         int qblocks) {
   // Let the next kernel (the product that reads xq) launch now: its CTAs can
   // set up and prefetch their weights while this grid runs; its own
   // grid-dependency wait still lasts until this grid has completed.
   pdl_launch_dependents();
   pdl_wait();
+  if (static_cast<int>(blockIdx.x) >= qblocks) {
+    expand_block<PERM>(job, static_cast<int64_t>(blockIdx.x) - qblocks);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
   if (m < M) {
@@ -275,23 +322,39 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) rms_norm_kernel(const void *
 
 }  // namespace
 
+cudaError_t launch_expand_weights(const ExpandJob &job, bool permuted, const LaunchCtx &ctx) {
+  if (job.words <= 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>(ceil_div(job.words, kExpandBlockWords)));
+  const dim3 block(32 * kRowsPerCta);
+  return permuted ? launch_k(expand_weights_kernel<true>, grid, block, 0, ctx, job)
+                  : launch_k(expand_weights_kernel<false>, grid, block, 0, ctx, job);
+}
+
 cudaError_t launch_quantize_act(const void *X, int x_kind, int64_t M, int64_t K, int8_t *xq,
-                                float *s, bool permuted, const LaunchCtx &ctx) {
+                                float *s, bool permuted, const LaunchCtx &ctx,
+                                const ExpandJob &expand) {
   if (M <= ctx.num_sms && K <= kRowMaxK) {  // few tokens: one CTA per row
     const dim3 grid(static_cast<unsigned>(M)), block(kRowThreads);
+    cudaError_t e;
     if (x_kind == kF32)
-      return permuted ? launch_k(quantize_row_kernel<kF32, true>, grid, block, 0, ctx, X, K, xq, s)
-                      : launch_k(quantize_row_kernel<kF32, false>, grid, block, 0, ctx, X, K, xq, s);
-    return permuted ? launch_k(quantize_row_kernel<kBF16, true>, grid, block, 0, ctx, X, K, xq, s)
-                    : launch_k(quantize_row_kernel<kBF16, false>, grid, block, 0, ctx, X, K, xq, s);
+      e = permuted ? launch_k(quantize_row_kernel<kF32, true>, grid, block, 0, ctx, X, K, xq, s)
+                   : launch_k(quantize_row_kernel<kF32, false>, grid, block, 0, ctx, X, K, xq, s);
+    else
+      e = permuted ? launch_k(quantize_row_kernel<kBF16, true>, grid, block, 0, ctx, X, K, xq, s)
+                   : launch_k(quantize_row_kernel<kBF16, false>, grid, block, 0, ctx, X, K, xq, s);
+    if (e != cudaSuccess) return e;
+    return launch_expand_weights(expand, permuted, ctx);
   }
-  const dim3 grid(static_cast<unsigned>(ceil_div(M, kRowsPerCta)));
+  const int64_t qblocks = ceil_div(M, kRowsPerCta);
+  const int64_t eblocks = expand.words > 0 ? ceil_div(expand.words, kExpandBlockWords) : 0;
+  const dim3 grid(static_cast<unsigned>(qblocks + eblocks));
   const dim3 block(32 * kRowsPerCta);
+  const int qb = static_cast<int>(qblocks);
   if (x_kind == kF32)
-    return permuted ? launch_k(quantize_act_kernel<kF32, true>, grid, block, 0, ctx, X, M, K, xq, s)
-                    : launch_k(quantize_act_kernel<kF32, false>, grid, block, 0, ctx, X, M, K, xq, s);
-  return permuted ? launch_k(quantize_act_kernel<kBF16, true>, grid, block, 0, ctx, X, M, K, xq, s)
-                  : launch_k(quantize_act_kernel<kBF16, false>, grid, block, 0, ctx, X, M, K, xq, s);
+    return permuted ? launch_k(quantize_act_kernel<kF32, true>, grid, block, 0, ctx, X, M, K, xq, s, expand, qb)
+                    : launch_k(quantize_act_kernel<kF32, false>, grid, block, 0, ctx, X, M, K, xq, s, expand, qb);
+  return permuted ? launch_k(quantize_act_kernel<kBF16, true>, grid, block, 0, ctx, X, M, K, xq, s, expand, qb)
+                  : launch_k(quantize_act_kernel<kBF16, false>, grid, block, 0, ctx, X, M, K, xq, s, expand, qb);
 }
 
 cudaError_t launch_rms_norm(const void *X, int x_kind, int64_t M, int64_t K, void *Y, int y_kind,
