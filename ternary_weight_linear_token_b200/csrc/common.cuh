@@ -221,6 +221,40 @@ __device__ __forceinline__ int quant_i8(float x, float s) {
   r = fminf(fmaxf(r, -127.0f), 127.0f);
   return static_cast<int>(__float_as_uint(__fadd_rn(r, kMagic)) - 0x4B400000u);
 }
+// quant_i8 for 16 activations of one row, for the throughput-bound
+// quantiser.  Within the quantiser's contract (finite x, s = 127 / max|x|
+// finite) |x * s| <= 127 * (1 + 2^-24) rounds to at most 127.0000077, so the
+// clamp never binds and is left out.  Adding 1.5 * 2^23 rounds v = x * s to
+// the nearest integer, ties to even, which the sum's low bits hold; r = that
+// sum minus 1.5 * 2^23 is the same integer as a float, and d = v - r is
+// exact, |d| <= 1/2.  A tie (|d| = 1/2) that went toward zero -- d has the
+// sign of v; with q != 0 that is the sign of q, with q = 0 (v = +-1/2) it
+// always is -- moves one step away.  Ties are rare: they are found by the
+// chunk's largest |d| and fixed in a branch.  Checked against the plain
+// definition for every float |v| <= 127.00002.  The three roundings are the
+// explicit _rn intrinsics, which the compiler never contracts: a fused
+// x * s + 1.5 * 2^23 would round the exact product instead of v and break
+// ties such as v = 63.5 (the paired f32x2 instructions did exactly that).
+__device__ __forceinline__ void quant16(const float (&x)[16], float s, int (&q)[16]) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
+  float d[16];
+  float dmax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float v = __fmul_rn(x[e], s);
+    const float t = __fadd_rn(v, kMagic);
+    q[e] = static_cast<int>(__float_as_uint(t) - 0x4B400000u);
+    d[e] = __fsub_rn(v, __fsub_rn(t, kMagic));
+    dmax = fmaxf(dmax, fabsf(d[e]));
+  }
+  if (dmax == 0.5f) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      if (fabsf(d[e]) == 0.5f && (q[e] == 0 || (d[e] > 0.0f) == (q[e] > 0)))
+        q[e] += d[e] > 0.0f ? 1 : -1;
+  }
+}
+
 // y = (float)acc * (gamma / s), then optionally ReLU^2.
 __device__ __forceinline__ float epilogue_value(int acc, float r, bool relu2) {
   float y = __fmul_rn(__int2float_rn(acc), r);
@@ -242,8 +276,9 @@ __device__ __forceinline__ uint32_t unpack_natural(uint32_t w, int j) {
 
 // Four int8 values into one 32-bit word, first value in the lowest byte.
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x0040u);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x0040u);
+  return __byte_perm(lo, hi, 0x5410u);
 }
 
 // 16 int8 activations of one 16-element group, stored in the order in which

@@ -122,8 +122,9 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
     const int64_t chunks = K / 16;
     const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(X) +
                                                       m * K * (KIND == kF32 ? 4 : 2));
-    // max |x| on the bit patterns: |x| of a float (or of a bf16) orders as an unsigned integer
-    uint32_t amax_bits = 0;
+    // max |x| on the bit patterns: |x| of a float (or of a bf16) orders as
+    // an unsigned integer; bf16 pairs go through the 16-bit SIMD max
+    uint32_t amax_bits = 0, amax_pair = 0;
     for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kInFlight) {
       uint4 raw[kInFlight][kWords];
 #pragma unroll
@@ -140,16 +141,15 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
             const uint32_t w[4] = {raw[i][j].x, raw[i][j].y, raw[i][j].z, raw[i][j].w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              if (KIND == kF32) {
+              if (KIND == kF32)
                 amax_bits = max(amax_bits, w[h] & 0x7FFFFFFFu);
-              } else {
-                amax_bits = max(amax_bits, (w[h] & 0x7FFFu) << 16);
-                amax_bits = max(amax_bits, w[h] & 0x7FFF0000u);
-              }
+              else
+                amax_pair = __vmaxu2(amax_pair, w[h] & 0x7FFF7FFFu);
             }
           }
         }
     }
+    if (KIND != kF32) amax_bits = max(amax_pair & 0xFFFFu, amax_pair >> 16) << 16;
     const float amax = warp_max(__uint_as_float(amax_bits));
     const float sm = act_scale(amax);
     for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kInFlight) {
@@ -179,8 +179,7 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
             }
           }
           int q[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) q[e] = quant_i8(v[e], sm);
+          quant16(v, sm, q);
           *reinterpret_cast<uint4 *>(xq + m * K + 16 * c) =
               PERM ? pack_permuted(q)
                    : make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),

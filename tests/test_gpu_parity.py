@@ -80,7 +80,10 @@ def _act_cases():
     yield "tiny", synth.config_inputs("tiny")["x"], "f32"
     yield "decode", synth.config_inputs("decode", weights=False)["x"], "bf16"
     yield "sweep_M32_K6912", synth.config_inputs("sweep", M=32, proj=3, weights=False)["x"], "bf16"
+    # bf16 rows whose products x * s round onto ties (v = +-63.5 hundreds of
+    # times): 200 rows take the warp-per-row kernel, 100 the CTA-per-row one
     yield "prefill_rows", synth.config_inputs("prefill", weights=False)["x"][:200], "bf16"
+    yield "prefill_rows_few", synth.config_inputs("prefill", weights=False)["x"][:100], "bf16"
     rng = np.random.default_rng(11)
     x = rng.standard_t(3, (7, 48)).astype(np.float32)
     x[2] = 0.0
