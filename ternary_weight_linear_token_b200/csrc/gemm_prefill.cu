@@ -35,27 +35,33 @@
 namespace bitnet {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                           // token rows per CTA
+constexpr int BN = 256;                           // features per accumulator
 constexpr int BK = 128;
-constexpr int kStages = 4;
 constexpr int kEpiWarps = 4;
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
 constexpr int kThreads = 32 * (kEpiWarps + 2);
 constexpr int kABytes = BM * BK;
-constexpr int kBBytes = BN * BK;
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * BN;
 constexpr int kStoreRows = 32;                    // epilogue staging block: 32 rows
 constexpr int kStoreCols = 64;                    // x 64 bf16 columns = 128-byte rows
 constexpr int kStoreBytes = kStoreRows * kStoreCols * 2;
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes +
-                              kEpiWarps * 2 * kStoreBytes + 256;
 
-// Instruction descriptor: s8 x s8 -> s32, both operands K-major, M=128, N=256.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) |
-                            ((BM >> 4) << 24);
+// One CTA: a 128 x 256 tile, A 16 KB + B 32 KB per stage, 4 stages.  A pair
+// (cta_group::2): a 256 x 256 tile, each CTA holding 128 token rows of A and
+// 128 feature rows of B, 16 KB + 16 KB per stage, 6 stages.
+template <bool PAIR> struct Cfg {
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kStageBytes = kABytes + kBRows * BK;
+  static constexpr int kTileM = PAIR ? 2 * BM : BM;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes +
+                                       kEpiWarps * 2 * kStoreBytes + 256;
+  // Instruction descriptor: s8 x s8 -> s32, both operands K-major, M = kTileM, N = 256.
+  static constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) |
+                                     ((kTileM >> 4) << 24);
+};
 
 struct PrefillParams {
   const float *s;
@@ -120,34 +126,41 @@ __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64
   }
 }
 
-template <int YK, bool RELU2, bool TMA_Y>
+// PAIR: launched as clusters of two CTAs; the first issues the pair MMAs for
+// both, each loads its own halves of A and B and writes its own 128 rows.
+template <int YK, bool RELU2, bool TMA_Y, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_y, const PrefillParams p) {
+  using C = Cfg<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *ring = smem;                                 // [kStages][A 16 KB | B 32 KB]
-  uint8_t *staging = ring + kStages * kStageBytes;      // [kEpiWarps][2][32 x 128 B]
+  uint8_t *ring = smem;                                   // [stages][A 16 KB | B]
+  uint8_t *staging = ring + C::kStages * C::kStageBytes;  // [kEpiWarps][2][32 x 128 B]
   uint64_t *full = reinterpret_cast<uint64_t *>(staging + kEpiWarps * 2 * kStoreBytes);
-  uint64_t *empty = full + kStages;
-  uint64_t *acc_full = empty + kStages;
+  uint64_t *empty = full + C::kStages;
+  uint64_t *acc_full = empty + C::kStages;
   uint64_t *acc_empty = acc_full + 2;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kblocks = static_cast<int>((p.K + BK - 1) / BK);
   const int tiles = p.m_tiles * p.n_tiles;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (warp == kWarpTma && lane == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], kEpiWarps);
+      mbar_init(&acc_empty[a], PAIR ? 2 * kEpiWarps : kEpiWarps);  // the pair's epilogues
     }
     fence_barrier_init();
     prefetch_tmap(&tmap_a);
@@ -155,15 +168,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (TMA_Y) prefetch_tmap(&tmap_y);
   }
   if (warp == kWarpMma) {
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<PAIR>(tmem_holder, kTmemCols);
+    tmem_relinquish<PAIR>();
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();  // both CTAs' barriers and TMEM exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  // Everything above overlaps the previous kernel; xq and s are its output.
+  // Everything above overlaps the previous kernel; xq, s and the int8
+  // weights are its output.
   pdl_wait();
   pdl_launch_dependents();
 
@@ -171,45 +186,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int32_t m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
+      for (int tile = unit; tile < tiles && ok; tile += units) {
+        const int32_t m0 = (tile / p.n_tiles) * C::kTileM + static_cast<int32_t>(rank) * BM;
+        const int32_t n0 = (tile % p.n_tiles) * BN + static_cast<int32_t>(rank) * C::kBRows;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages;
-          if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, p.status)) {
+          const int s = it % C::kStages;
+          if (it >= C::kStages &&
+              !mbar_wait<PAIR>(&empty[s], ((it / C::kStages) - 1) & 1, p.status)) {
             ok = false;
             break;
           }
-          uint8_t *stage = ring + s * kStageBytes;
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          tma_load_2d(stage, &tmap_a, kb * BK, m0, &full[s]);
-          tma_load_2d(stage + kABytes, &tmap_b, kb * BK, n0, &full[s]);
+          uint8_t *stage = ring + s * C::kStageBytes;
+          if (PAIR) {
+            // both CTAs' halves complete on the first CTA's barrier
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+            const uint32_t bar0 = mapa_shared(&full[s], 0);
+            tma_load_2d_pair(stage, &tmap_a, kb * BK, m0, bar0);
+            tma_load_2d_pair(stage + kABytes, &tmap_b, kb * BK, n0, bar0);
+          } else {
+            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+            tma_load_2d(stage, &tmap_a, kb * BK, m0, &full[s]);
+            tma_load_2d(stage + kABytes, &tmap_b, kb * BK, n0, &full[s]);
+          }
         }
       }
     }
   } else if (warp == kWarpMma) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       uint32_t it = 0;
       bool ok = true;
       int tl = 0;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tl) {
+      for (int tile = unit; tile < tiles && ok; tile += units, ++tl) {
         const int acc = tl & 1;
-        if (tl >= 2 && !mbar_wait(&acc_empty[acc], ((tl >> 1) - 1) & 1, p.status)) break;
+        if (tl >= 2 && !mbar_wait<PAIR>(&acc_empty[acc], ((tl >> 1) - 1) & 1, p.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const int s = it % kStages;
-          ok = mbar_wait(&full[s], (it / kStages) & 1, p.status);
+          const int s = it % C::kStages;
+          ok = mbar_wait<PAIR>(&full[s], (it / C::kStages) & 1, p.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(ring + s * kStageBytes);
+          const uint32_t a_base = smem_u32(ring + s * C::kStageBytes);
           const uint32_t b_base = a_base + kABytes;
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk)
-            mma_i8(d, smem_desc_sw128(a_base + 32 * kk), smem_desc_sw128(b_base + 32 * kk), kIdesc,
-                   (kb | kk) != 0 ? 1u : 0u);
-          mma_commit(&empty[s]);
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_base + 32 * kk);
+            const uint64_t bd = smem_desc_sw128(b_base + 32 * kk);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (PAIR)
+              mma_i8_pair(d, ad, bd, C::kIdesc, accum);
+            else
+              mma_i8(d, ad, bd, C::kIdesc, accum);
+          }
+          if (PAIR)
+            mma_commit_pair(&empty[s]);
+          else
+            mma_commit(&empty[s]);
         }
-        mma_commit(&acc_full[acc]);
+        if (PAIR)
+          mma_commit_pair(&acc_full[acc]);
+        else
+          mma_commit(&acc_full[acc]);
       }
     }
   } else {
@@ -218,12 +255,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float gamma = *p.gamma;
     const bool vec_ok = (YK == kBF16) ? (p.N % 8 == 0) : (p.N % 4 == 0);
     uint8_t *my_stage = staging + q * 2 * kStoreBytes;
+    // the accumulator is released to the pair's first CTA (its MMA reuses it)
+    const uint32_t acc_empty0_a = PAIR ? mapa_shared(&acc_empty[0], 0) : 0u;
+    const uint32_t acc_empty0_b = PAIR ? mapa_shared(&acc_empty[1], 0) : 0u;
     int tl = 0, stores = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tl) {
+    for (int tile = unit; tile < tiles; tile += units, ++tl) {
       const int acc = tl & 1;
-      if (!mbar_wait(&acc_full[acc], (tl >> 1) & 1, p.status)) break;
+      if (!mbar_wait<PAIR>(&acc_full[acc], (tl >> 1) & 1, p.status)) break;
       tc_fence_after();
-      const int64_t m_base = static_cast<int64_t>(tile / p.n_tiles) * BM + q * 32;
+      const int64_t m_base = static_cast<int64_t>(tile / p.n_tiles) * C::kTileM +
+                             static_cast<int64_t>(rank) * BM + q * 32;
       const int64_t m = m_base + lane;
       const int64_t n0 = static_cast<int64_t>(tile % p.n_tiles) * BN;
       const float r = (m < p.M) ? __fdiv_rn(gamma, p.s[m]) : 0.0f;
@@ -248,7 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (cb == BN / kStoreCols - 1 && half == 1) {  // accumulator fully read
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[acc]);
+              if (lane == 0) {
+                if (PAIR)
+                  mbar_arrive_remote(acc ? acc_empty0_b : acc_empty0_a);
+                else
+                  mbar_arrive(&acc_empty[acc]);
+              }
             }
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {  // 8 columns = 16 bytes per chunk, swizzled
@@ -283,14 +329,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (lane == 0) {
+          if (PAIR)
+            mbar_arrive_remote(acc ? acc_empty0_b : acc_empty0_a);
+          else
+            mbar_arrive(&acc_empty[acc]);
+        }
       }
     }
     if (TMA_Y && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) tmem_dealloc(tmem_base, kTmemCols);
+  // the other CTA of a pair may still be signalled by (or signal) this one's
+  // barriers and TMEM until both are done
+  if (PAIR) cluster_sync();
+  if (warp == kWarpMma) tmem_dealloc<PAIR>(tmem_base, kTmemCols);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -321,26 +375,36 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YK, bool RELU2, bool TMA_Y>
+template <int YK, bool RELU2, bool TMA_Y, bool PAIR>
 cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
                const PrefillParams &p, const LaunchCtx &ctx) {
-  auto kern = prefill_kernel<YK, RELU2, TMA_Y>;
+  using C = Cfg<PAIR>;
+  auto kern = prefill_kernel<YK, RELU2, TMA_Y, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+                                       static_cast<int>(C::kSmemBytes));
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-  const dim3 grid(static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms));
-  return launch_k(kern, grid, dim3(kThreads), kSmemBytes, ctx, ta, tb, ty, p);
+  if (!PAIR) {
+    const dim3 grid(static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms));
+    return launch_k(kern, grid, dim3(kThreads), C::kSmemBytes, ctx, ta, tb, ty, p);
+  }
+  const int64_t pairs = ctx.num_sms / 2;
+  const dim3 grid(static_cast<unsigned>(2 * (tiles < pairs ? tiles : pairs)));
+  return launch_k_cluster(kern, grid, dim3(kThreads), C::kSmemBytes, 2u, ctx, ta, tb, ty, p);
 }
 
+template <bool PAIR>
 cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, bool tma_y,
                  const PrefillParams &p, int y_kind, bool relu2, const LaunchCtx &ctx) {
-  if (y_kind == kI32) return go<kI32, false, false>(ta, tb, ty, p, ctx);
+  if (y_kind == kI32) return go<kI32, false, false, PAIR>(ta, tb, ty, p, ctx);
   if (y_kind == kF32)
-    return relu2 ? go<kF32, true, false>(ta, tb, ty, p, ctx) : go<kF32, false, false>(ta, tb, ty, p, ctx);
+    return relu2 ? go<kF32, true, false, PAIR>(ta, tb, ty, p, ctx)
+                 : go<kF32, false, false, PAIR>(ta, tb, ty, p, ctx);
   if (tma_y)
-    return relu2 ? go<kBF16, true, true>(ta, tb, ty, p, ctx) : go<kBF16, false, true>(ta, tb, ty, p, ctx);
-  return relu2 ? go<kBF16, true, false>(ta, tb, ty, p, ctx) : go<kBF16, false, false>(ta, tb, ty, p, ctx);
+    return relu2 ? go<kBF16, true, true, PAIR>(ta, tb, ty, p, ctx)
+                 : go<kBF16, false, true, PAIR>(ta, tb, ty, p, ctx);
+  return relu2 ? go<kBF16, true, false, PAIR>(ta, tb, ty, p, ctx)
+               : go<kBF16, false, false, PAIR>(ta, tb, ty, p, ctx);
 }
 
 }  // namespace
@@ -358,11 +422,13 @@ size_t prefill_weight_bytes(int64_t N, int64_t K) { return static_cast<size_t>(N
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                            void *Y, int y_kind, const LaunchCtx &ctx) {
+  // more than one 128-token block: CTA pairs on 256-token tiles
+  const bool pair = M > BM && ctx.num_sms >= 2;
   CUtensorMap ta, tb;
   if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                    static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                   static_cast<uint64_t>(K), BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint64_t>(K), BK, pair ? BN / 2 : BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   PrefillParams p;
   p.s = s;
@@ -372,7 +438,7 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
   p.M = M;
   p.N = N;
   p.K = K;
-  p.m_tiles = static_cast<int>(ceil_div(M, BM));
+  p.m_tiles = static_cast<int>(ceil_div(M, pair ? 2 * BM : BM));
   p.n_tiles = static_cast<int>(ceil_div(N, BN));
   // bf16 output with 16-byte rows goes out through TMA tensor stores
   CUtensorMap ty;
@@ -381,7 +447,8 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                                  static_cast<uint64_t>(N) * 2, kStoreCols, kStoreRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   if (!tma_y) ty = ta;  // unused by the direct-store kernels
-  return go_y(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+  return pair ? go_y<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx)
+              : go_y<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet
