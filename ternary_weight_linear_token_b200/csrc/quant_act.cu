@@ -96,6 +96,62 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) expand_weights_kernel(const 
   expand_block<PERM>(job, blockIdx.x);
 }
 
+// A bf16 row of up to 32 * kRegChunks 16-element chunks, one warp: the whole
+// row is loaded into registers with every load issued up front, so it costs
+// one round trip to memory, where the two-pass loop below costs one per pass
+// and load round.
+constexpr int kRegChunks = 6;
+template <bool PERM>
+__device__ __forceinline__ void quantize_row_resident(const uint4 *row, int chunks, int lane,
+                                                      int8_t *out, float *s_out) {
+  uint4 raw[kRegChunks][2];
+#pragma unroll
+  for (int i = 0; i < kRegChunks; ++i) {
+    const int c = lane + 32 * i;
+    if (c < chunks) {
+      raw[i][0] = row[2 * c];
+      raw[i][1] = row[2 * c + 1];
+    } else {
+      raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  uint32_t amax_pair = 0;  // 16-bit SIMD max of |x| bit patterns (zeros past the row)
+#pragma unroll
+  for (int i = 0; i < kRegChunks; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      amax_pair = __vmaxu2(amax_pair, raw[i][j].x & 0x7FFF7FFFu);
+      amax_pair = __vmaxu2(amax_pair, raw[i][j].y & 0x7FFF7FFFu);
+      amax_pair = __vmaxu2(amax_pair, raw[i][j].z & 0x7FFF7FFFu);
+      amax_pair = __vmaxu2(amax_pair, raw[i][j].w & 0x7FFF7FFFu);
+    }
+  const uint32_t amax_bits = max(amax_pair & 0xFFFFu, amax_pair >> 16) << 16;
+  const float sm = act_scale(warp_max(__uint_as_float(amax_bits)));
+#pragma unroll
+  for (int i = 0; i < kRegChunks; ++i) {
+    const int c = lane + 32 * i;
+    if (c < chunks) {
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t w[4] = {raw[i][j].x, raw[i][j].y, raw[i][j].z, raw[i][j].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          v[8 * j + 2 * h] = __uint_as_float(w[h] << 16);
+          v[8 * j + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+        }
+      }
+      int q[16];
+      quant16(v, sm, q);
+      *reinterpret_cast<uint4 *>(out + 16 * c) =
+          PERM ? pack_permuted(q)
+               : make_uint4(pack4(q[0], q[1], q[2], q[3]), pack4(q[4], q[5], q[6], q[7]),
+                            pack4(q[8], q[9], q[10], q[11]), pack4(q[12], q[13], q[14], q[15]));
+    }
+  }
+  if (lane == 0) *s_out = sm;
+}
+
 // Blocks [0, qblocks) quantise 8 token rows each; later blocks expand the
 // weights of `job` (none when job.words == 0).
 template <int KIND, bool PERM>
@@ -115,7 +171,11 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) quantize_act_kernel(const vo
   }
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
-  if (m < M) {
+  if (m < M && KIND == kBF16 && K <= 32 * 16 * kRegChunks) {
+    quantize_row_resident<PERM>(
+        reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(X) + m * K),
+        static_cast<int>(K / 16), lane, xq + m * K, s + m);
+  } else if (m < M) {
     // 16-element steps per lane per round: the raw words stay in registers
     constexpr int kInFlight = KIND == kF32 ? 2 : 4;
     constexpr int kWords = KIND == kF32 ? 4 : 2;  // uint4 per 16 elements

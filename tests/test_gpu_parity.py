@@ -121,6 +121,9 @@ SHAPES = [
     # 4..8 tokens quantised inside the mma.sync kernel: one K step (fewer than
     # the warps), N below one 8-row block, an odd step count, the largest K
     (4, 7, 64), (7, 9, 192), (4, 2000, 1088), (5, 1201, 4096), (8, 2560, 4160),
+    # more than 148 tokens: the quantiser's warp-per-row kernel keeps a bf16
+    # row in registers up to K = 3072 and loops in two passes above it
+    (200, 24, 3072), (150, 24, 3136), (160, 40, 6912),
 ]
 
 
