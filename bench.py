@@ -172,6 +172,30 @@ class Workload:
     bound = "hbm"
 
 
+def workload_identity(workload: str, sweep_m: int = 8, layers: int = 30) -> dict:
+    """What a workload is (shapes, distributions, dtypes), shared by both arms' JSON lines."""
+    if workload == "decode":
+        return {"workload": "decode GEMV M=1 K=2560 N=2560, bf16 activations N(0,1) with 0.1% "
+                            "x20 outliers, absmean ternary weights from N(0,0.02), bf16 out",
+                "M": 1, "K": 2560, "N": 2560, "x_dtype": "bf16", "y_dtype": "bf16"}
+    if workload == "sweep":
+        return {"workload": f"decode sweep M={sweep_m}: one decoder layer's BitLinears, qkv "
+                            "2560->3840, o 2560->2560, up 2560->6912 + ReLU^2, down 6912->2560; "
+                            "Student-t(3) bf16 activations, absmean ternary weights from "
+                            "N(0,0.02), bf16 out",
+                "M": sweep_m, "x_dtype": "bf16", "y_dtype": "bf16"}
+    if workload == "prefill":
+        return {"workload": "prefill GEMM M=4096 K=2560 N=6912, bf16 activations N(0,1) "
+                            "per-token absmax int8, ternary weights from N(0,0.02), int32 "
+                            "accumulation, bf16 out",
+                "M": 4096, "K": 2560, "N": 6912, "x_dtype": "bf16", "y_dtype": "bf16"}
+    if workload == "chain":
+        return {"workload": f"{layers}-layer decode chain, M=1, per layer qkv 2560->3840, "
+                            "o 2560->2560, up 2560->6912 + ReLU^2, down 6912->2560, rms norm",
+                "M": 1, "layers": layers, "x_dtype": "bf16", "y_dtype": "bf16"}
+    raise ValueError(workload)
+
+
 def make_decode(tw, torch, dev, l2_bytes):
     import synth
     d = synth.config_inputs("decode")
@@ -191,9 +215,7 @@ def make_decode(tw, torch, dev, l2_bytes):
     return dict(
         step=step, kernel_step=step, units_per_step=wbytes, unit="GB/s", scale=1e-9, bound="hbm",
         launches_per_step=1, X=X, Y=Y, rotate=R, extra=dict(packed=copies, gamma=gamma),
-        config={"workload": "decode GEMV M=1 K=2560 N=2560, bf16 activations N(0,1) with 0.1% "
-                            "x20 outliers, absmean ternary weights from N(0,0.02), bf16 out",
-                "M": 1, "K": 2560, "N": 2560, "x_dtype": "bf16", "y_dtype": "bf16",
+        config={**workload_identity("decode"),
                 "l2": f"inputs larger than L2: {R} rotating weight copies, "
                       f"{R * wbytes / 1e6:.0f} MB >= 3x L2",
                 "timing": "CUDA graph of the timed steps, programmatic dependent launch, "
@@ -235,10 +257,7 @@ def make_sweep(tw, torch, dev, l2_bytes, M=8):
     return dict(
         step=step, kernel_step=step, units_per_step=wbytes, unit="GB/s", scale=1e-9, bound="hbm",
         launches_per_step=launches, X=projs[0]["X"], Y=projs[3]["Y"], rotate=R,
-        config={"workload": f"decode sweep M={M}: one decoder layer's BitLinears, qkv 2560->3840, "
-                            "o 2560->2560, up 2560->6912 + ReLU^2, down 6912->2560; Student-t(3) "
-                            "bf16 activations, absmean ternary weights from N(0,0.02), bf16 out",
-                "M": M, "x_dtype": "bf16", "y_dtype": "bf16",
+        config={**workload_identity("sweep", sweep_m=M),
                 "l2": f"inputs larger than L2: {R} rotating copies of the layer's weights, "
                       f"{R * wbytes / 1e6:.0f} MB >= 3x L2",
                 "timing": "CUDA graph of the timed steps, programmatic dependent launch, "
@@ -283,10 +302,7 @@ def make_prefill(tw, torch, dev, l2_bytes):
         step=step, kernel_step=None, quant_step=quant_step, units_per_step=ops, unit="TOPS",
         scale=1e-12,
         bound="tensor", launches_per_step=2, rotate=R, X=X0, Y=Ys[0],
-        config={"workload": "prefill GEMM M=4096 K=2560 N=6912, bf16 activations N(0,1) "
-                            "per-token absmax int8, ternary weights from N(0,0.02), int32 "
-                            "accumulation, bf16 out",
-                "M": M, "K": K, "N": N, "x_dtype": "bf16", "y_dtype": "bf16",
+        config={**workload_identity("prefill"),
                 "l2": f"inputs larger than L2: {R} rotating input/output sets",
                 "timing": "CUDA graph; step = activation quantiser (the weights' expansion to "
                           "int8 scratch runs in the same launch) + tcgen05 kernel"},
@@ -317,9 +333,7 @@ def make_chain(tw, torch, dev, l2_bytes, layers=30, persistent=False):
     return dict(
         step=step, kernel_step=None, units_per_step=wbytes, unit="GB/s", scale=1e-9, bound="hbm",
         launches_per_step=chain.launches_per_token(), rotate=1, X=chain.x_in, Y=chain.outs[-1][4],
-        config={"workload": f"{layers}-layer decode chain, M=1, per layer qkv 2560->3840, "
-                            "o 2560->2560, up 2560->6912 + ReLU^2, down 6912->2560, rms norm",
-                "M": 1, "layers": layers, "x_dtype": "bf16", "y_dtype": "bf16",
+        config={**workload_identity("chain", layers=layers),
                 "l2": f"inputs larger than L2: {wbytes / 1e6:.0f} MB of packed weights per token",
                 "mode": ("one persistent launch per token (bitnet_decode_chain)" if persistent
                          else "one launch per projection and per normalisation"),
@@ -333,7 +347,7 @@ MAKERS = {"decode": make_decode, "prefill": make_prefill, "chain": make_chain,
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_sample(workload: str, budget_s: float):
+def oracle_sample(workload: str, budget_s: float, sweep_m: int = 8):
     """Time the plain C oracle on a bounded sample of the workload on the host
     cores.  Returns (value, unit, cores, sample description, seconds)."""
     import synth
@@ -354,9 +368,26 @@ def oracle_sample(workload: str, budget_s: float):
         ops = 2 * rows * n * d["N"] * d["K"]
         return ops / dt * 1e-12, "TOPS", R.num_threads(), f"{n * rows} token rows x N=6912 x K=2560", dt
     if workload in ("chain", "sweep"):
-        d = synth.config_inputs("sweep", M=1, proj=2)
-    else:
-        d = synth.config_inputs("decode")
+        # one decoder layer: the four projections at the workload's tokens per call
+        M = sweep_m if workload == "sweep" else 1
+        projs = []
+        for p in range(4):
+            d = synth.config_inputs("sweep", M=M, proj=p)
+            packed, gamma = R.quantize_weights(d["W"])
+            projs.append((d, packed, gamma))
+        layer_bytes = sum(packed.size for _, packed, _ in projs)
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            for d, packed, gamma in projs:
+                R.bitlinear(d["x"], packed, gamma, d["N"], relu2=d["relu2"])
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return (n * layer_bytes / dt * 1e-9, "GB/s", R.num_threads(),
+                f"{n} decoder layers (qkv, o, up + ReLU^2, down) at M={M}", dt)
+    d = synth.config_inputs("decode")
     packed, gamma = R.quantize_weights(d["W"])
     t0 = time.perf_counter()
     n = 0
@@ -376,14 +407,14 @@ def run_reference(args, world, rank):
         return 0
     per_step = max(0.02, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(args.workload, per_step / 4)
+        oracle_sample(args.workload, per_step / 4, args.sweep_m)
     tot_units = 0.0
     t0 = time.perf_counter()
     cores = 1
     sample = ""
     unit = "GB/s"
     for _ in range(args.steps):
-        v, unit, cores, sample, dt = oracle_sample(args.workload, per_step)
+        v, unit, cores, sample, dt = oracle_sample(args.workload, per_step, args.sweep_m)
         tot_units += v * dt
     dt = time.perf_counter() - t0
     value = tot_units / dt
@@ -391,7 +422,9 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
             "data": "synthetic",
-            "config": {"workload": args.workload + " (oracle on host cores, bounded sample per step)"},
+            "config": {**workload_identity(args.workload, sweep_m=args.sweep_m),
+                       "timing": "the oracle (plain C) on the host cores, a bounded sample of "
+                                 "the workload per step, scaled to the metric's unit"},
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": f"per step ~{per_step:.2f} s of: {sample}"},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -533,7 +566,7 @@ def main():
     status = tw.bitnet_get_device_status(stream)
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        v, unit, cores, sample, dt = oracle_sample(args.workload, args.cpu_seconds)
+        v, unit, cores, sample, dt = oracle_sample(args.workload, args.cpu_seconds, args.sweep_m)
         cpu = {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
                "sample": f"{sample} in {dt:.1f} s"}
     if rank == 0:

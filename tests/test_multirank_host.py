@@ -53,3 +53,27 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "--gpus", "2", "--steps", "1", "--warmup", "1"], env=env,
                        capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_line_matches_our_arm():
+    """Rank 0 of the reference arm prints one JSON line carrying the contract's
+    keys, the same metric and workload identity as our arm, and its own
+    description as cpu_baseline and e2e (no host<->device bytes)."""
+    import json
+    import bench
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "1"], capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert d["warmup"] >= 3 and d["steps"] == 1 and d["n_gpus"] == 1
+    ident = bench.workload_identity("decode")
+    assert {k: d["config"][k] for k in ident} == ident
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
