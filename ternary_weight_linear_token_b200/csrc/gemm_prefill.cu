@@ -29,6 +29,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -47,6 +49,7 @@ constexpr int kTmemCols = 2 * BN;
 constexpr int kStoreRows = 32;                    // epilogue staging block: 32 rows
 constexpr int kStoreCols = 64;                    // x 64 bf16 columns = 128-byte rows
 constexpr int kStoreBytes = kStoreRows * kStoreCols * 2;
+constexpr int kMaxDevices = 64;
 
 // One CTA: a 128 x 256 tile, A 16 KB + B 32 KB per stage, 4 stages.  A pair
 // (cta_group::2): a 256 x 256 tile, each CTA holding 128 token rows of A and
@@ -388,7 +391,35 @@ cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &
     const dim3 grid(static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms));
     return launch_k(kern, grid, dim3(kThreads), C::kSmemBytes, ctx, ta, tb, ty, p);
   }
-  const int64_t pairs = ctx.num_sms / 2;
+  // as many pairs as the device can hold at once (asked once per device); none: the
+  // caller runs single CTAs
+  static std::atomic<int> resident[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int most = resident[dev].load(std::memory_order_relaxed);
+  if (most == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (ctx.num_sms / 2)));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    most = n > 0 ? n : -1;
+    resident[dev].store(most, std::memory_order_relaxed);
+  }
+  if (most < 1) return cudaErrorInvalidClusterSize;
+  int64_t pairs = ctx.num_sms / 2;
+  if (pairs > most) pairs = most;
   const dim3 grid(static_cast<unsigned>(2 * (tiles < pairs ? tiles : pairs)));
   return launch_k_cluster(kern, grid, dim3(kThreads), C::kSmemBytes, 2u, ctx, ta, tb, ty, p);
 }
@@ -422,14 +453,6 @@ size_t prefill_weight_bytes(int64_t N, int64_t K) { return static_cast<size_t>(N
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
                            void *Y, int y_kind, const LaunchCtx &ctx) {
-  // more than one 128-token block: CTA pairs on 256-token tiles
-  const bool pair = M > BM && ctx.num_sms >= 2;
-  CUtensorMap ta, tb;
-  if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                   static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                   static_cast<uint64_t>(K), BK, pair ? BN / 2 : BN, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
   PrefillParams p;
   p.s = s;
   p.gamma = gamma;
@@ -438,17 +461,31 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
   p.M = M;
   p.N = N;
   p.K = K;
-  p.m_tiles = static_cast<int>(ceil_div(M, pair ? 2 * BM : BM));
   p.n_tiles = static_cast<int>(ceil_div(N, BN));
+  CUtensorMap ta, tb, ty;
+  if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                   static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   // bf16 output with 16-byte rows goes out through TMA tensor stores
-  CUtensorMap ty;
   const bool tma_y = y_kind == kBF16 && N % 8 == 0 &&
                      make_map_2d(&ty, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
                                  static_cast<uint64_t>(N) * 2, kStoreCols, kStoreRows,
                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   if (!tma_y) ty = ta;  // unused by the direct-store kernels
-  return pair ? go_y<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx)
-              : go_y<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+  // more than one 128-token block: CTA pairs on 256-token tiles
+  if (M > BM && ctx.num_sms >= 2) {
+    if (!make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                     static_cast<uint64_t>(K), BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    p.m_tiles = static_cast<int>(ceil_div(M, 2 * BM));
+    const cudaError_t e = go_y<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+    if (e != cudaErrorInvalidClusterSize) return e;  // else: no pair fits, single CTAs
+  }
+  if (!make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                   static_cast<uint64_t>(K), BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  p.m_tiles = static_cast<int>(ceil_div(M, BM));
+  return go_y<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet
