@@ -4,7 +4,7 @@
 // The activations arrive quantised (bitnet_quantize_act, int8 in the K order
 // of the byte-permute weight unpack, one 16-byte chunk per packed word) and
 // are staged in shared memory by one bulk copy per token when they fit
-// beside the weights (else read from L2 in the loop).  The
+// beside the weights (else read from L2 in the loop, one K step ahead).  The
 // grid has one CTA per SM, each owning a contiguous range of 8-row blocks of
 // the weights (2 to 8 blocks), so the grid balances to within 8 rows; the
 // CTA's packed rows arrive by bulk copies into padded shared-memory rows,
@@ -154,18 +154,25 @@ __global__ void __launch_bounds__(kThreads, 1) mmv_kernel(const MmvParams p) {
     for (int a = 0; a < MT16; ++a) c[b][a][0] = c[b][a][1] = c[b][a][2] = c[b][a][3] = 0;
 
   if (weights_ok) {
-    for (int st = st0; st < st1; ++st) {
+    // A: 16-byte activation chunks of this lane's tokens (zero past M); the
+    // next step's chunks are loaded before this step's MMAs, so one load
+    // latency overlaps one step of math
+    uint4 xa[MT16][2], xn[MT16][2];
+    auto load_x = [&](int st, uint4 (&dst)[MT16][2]) {
       const int word = 4 * st + tq;
-      // A: 16-byte activation chunks of this lane's tokens (zero past M)
-      uint4 xa[MT16][2];
 #pragma unroll
       for (int a = 0; a < MT16; ++a)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int tok = 16 * a + 8 * h + g;
-          xa[a][h] = tok < p.M ? *reinterpret_cast<const uint4 *>(xsrc + static_cast<size_t>(tok) * p.K + 16 * word)
-                               : make_uint4(0u, 0u, 0u, 0u);
+          dst[a][h] = tok < p.M ? *reinterpret_cast<const uint4 *>(xsrc + static_cast<size_t>(tok) * p.K + 16 * word)
+                                : make_uint4(0u, 0u, 0u, 0u);
         }
+    };
+    if (st0 < st1) load_x(st0, xa);
+    for (int st = st0; st < st1; ++st) {
+      const int word = 4 * st + tq;
+      if (st + 1 < st1) load_x(st + 1, xn);
 #pragma unroll
       for (int b = 0; b < kMaxBlocks; ++b) {
         if (b < nb) {
@@ -178,6 +185,11 @@ __global__ void __launch_bounds__(kThreads, 1) mmv_kernel(const MmvParams p) {
             mma_16832(c[b][a], xa[a][0].z, xa[a][1].z, xa[a][0].w, xa[a][1].w, b2, b3);
           }
         }
+      }
+#pragma unroll
+      for (int a = 0; a < MT16; ++a) {
+        xa[a][0] = xn[a][0];
+        xa[a][1] = xn[a][1];
       }
     }
   }
