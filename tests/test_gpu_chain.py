@@ -158,15 +158,18 @@ def test_decode_chain_matches_per_launch_chain(tw):
 
 def test_decode_chain_bounded_wait_reports_timeout(tw):
     """A wait that never completes gives up (about 2 s) and is reported, with
-    no fault: the finished-CTA counter in a zero-filled workspace is set to 1,
-    so the count CTA 0 waits for at the end never appears.  The links computed
-    before that are still right, the device status is BITNET_ERR_TIMEOUT, and
-    the launch counter is not advanced (zero the workspace again after a
-    timeout, as the header says)."""
+    no fault: the finished-CTA counter in a zero-filled workspace starts at
+    2^30, above the count CTA 0 waits for at the end (the number of CTAs), and
+    only grows, so that count never appears.  (A start of 1 would not do: the
+    count then passes through the awaited value just before the last CTA
+    counts itself out, and CTA 0 may see it.)  The links computed before that
+    are still right, the device status is BITNET_ERR_TIMEOUT, and the launch
+    counter is not advanced (zero the workspace again after a timeout, as the
+    header says)."""
     steps, Ws = build_chain(tw, SHAPES_A[:2], 31)
     arr = tw.bitnet_decode_chain_steps(steps)
     ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
-    ws.view(torch.int32)[32] = 1  # byte 128: the finished-CTA counter
+    ws.view(torch.int32)[32] = 1 << 30  # byte 128: the finished-CTA counter
     assert tw.bitnet_get_device_status() == tw.OK
     x0 = x0_bits(SHAPES_A[0][1], 7)
     tw.bitnet_decode_chain(arr, bf16_t(x0), ws)
