@@ -7,25 +7,32 @@
 // The int8 weights come from the packed ones by a coalesced expansion pass
 // beforehand (launched with the activation quantiser: 4.4 MB in, 17.7 MB out
 // for 6912 x 2560), in the K order of the activations.
-// prefill_kernel: persistent, one CTA per SM, output tiles of 128 tokens x
-//               256 features taken round-robin; K in 128-byte stages.
-//     warp 4    TMA producer: the xq tile [128 x 128 B] and the int8 weight
-//               tile [256 x 128 B], both 128-byte swizzled, into a 4-stage ring.
-//     warp 5    allocates 512 TMEM columns (two 256-column accumulators); one
-//               lane issues 4 MMAs (M=128, N=256, K=32) per stage and commits
-//               them to the barrier that frees the stage, and, after a tile's
-//               last stage, to the accumulator-full barrier.
-//     warps 0-3 epilogue: tcgen05.ld of the finished accumulator, y = acc *
-//               (gamma / s_m), optional ReLU^2; bf16 output goes through a
-//               128-byte-swizzled shared-memory staging block (32 rows x 64
-//               columns per warp, double-buffered) and a TMA tensor store,
-//               so HBM sees whole lines; then the accumulator is released,
-//               so tile i's epilogue overlaps tile i+1's MMAs.
+// prefill_kernel: persistent, K in 128-byte stages, two 256-column int32
+// accumulators in TMEM (512 columns) so that tile i's epilogue overlaps tile
+// i+1's MMAs.  Two forms:
+//   CTA pairs (M > 128; clusters of two CTAs on two SMs, cta_group::2):
+//     output tiles of 256 tokens x 256 features taken round-robin by the
+//     pairs.  Each CTA's TMA warp (4) loads its own 128 token rows of xq and
+//     its own 128 feature rows of the int8 weights (128-byte swizzled, 6-stage
+//     ring of 16 + 16 KB); both CTAs' bytes complete on the first CTA's
+//     barrier (.cta_group::2 loads, no multicast).  One lane of the first
+//     CTA's warp 5 issues 4 pair MMAs (M=256, N=256, K=32) per stage, A and
+//     B read from both CTAs' shared memory at the same offsets, and commits
+//     with .multicast::cluster to both CTAs' stage-empty and
+//     accumulator-full barriers.  D rows 0-127 land in the first CTA's TMEM,
+//     128-255 in the second's.
+//   single CTAs (M <= 128): tiles of 128 tokens x 256 features, a 4-stage
+//     ring of 16 + 32 KB, M=128 MMAs.
+//   warps 0-3 (every CTA) epilogue: tcgen05.ld of its 128 accumulator rows,
+//     y = acc * (gamma / s_m), optional ReLU^2; bf16 output goes through a
+//     128-byte-swizzled shared-memory staging block (32 rows x 64 columns per
+//     warp, double-buffered) and a TMA tensor store, so HBM sees whole
+//     lines; then the accumulator is released (in a pair, with a
+//     cluster-scope arrive on the first CTA's barrier: 8 arrivals).
 // Expanding in HBM first keeps shared memory for the tensor core's operands
-// only: per 128-byte K stage it carries the TMA writes (48 KB) and the
-// operand reads (48 KB); expanding inside the kernel added the packed reads
-// and the expanded stores (40 KB more) and bounded the kernel by shared-memory
-// bandwidth.  Every wait is bounded (see common.cuh).
+// only; the pair form halves each SM's share of them to 32 KB of TMA writes
+// and 32 KB of operand reads per stage, under what the MMAs take.  Every wait
+// is bounded (see common.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
