@@ -316,9 +316,41 @@ def pin_bf16(R):
     assert [int(v) for v in R.to_bf16(vals)] == want
 
 
+# ------------------------------------------------------------------ rms norm (chain glue)
+def _rms_norm_exact(row):
+    """x / sqrt(mean(x^2) + 1e-6) in 50-digit decimal arithmetic, with the
+    stand-in's epsilon taken as the double nearest 1e-6."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 50
+    xs = [Decimal(float(v)) for v in row]
+    ms = sum(v * v for v in xs) / len(xs) + Decimal(1e-6)
+    inv = 1 / ms.sqrt()
+    return [float(v * inv) for v in xs]
+
+
+def pin_rms_norm(R):
+    """The weightless per-token RMS normalisation that stands in for the
+    model card's subln (模型详情 -> 架构; no formula on the pages), against
+    high-precision values, within 2 fp32 ulps: rows of 1e-3 (where the
+    epsilon doubles the mean square), a lone 1 among zeros (mean over K, not
+    the sum), 3 and 4, a zero row (stays zero), and a random row whose
+    output mean square is 1."""
+    rows = [np.full(4, 1e-3, dtype=np.float32), np.array([1, 0, 0, 0], dtype=np.float32),
+            np.array([3, 4], dtype=np.float32), np.zeros(3, dtype=np.float32),
+            np.random.default_rng(5).standard_normal(64).astype(np.float32)]
+    for row in rows:
+        got = R.rms_norm(row[None, :])[0]
+        want = np.array(_rms_norm_exact(row))
+        tol = 2 * np.spacing(np.abs(want).astype(np.float32)).astype(np.float64)
+        assert np.all(np.abs(got.astype(np.float64) - want) <= tol), (row[:4], got[:4], want[:4])
+    big = rows[-1]
+    y = R.rms_norm(big[None, :])[0].astype(np.float64)
+    assert abs(np.mean(y * y) - 1.0) < 1e-5
+
+
 ALL_PINS = [
     pin_code_table, pin_weight_boundaries, pin_weight_special, pin_gamma_exact,
     pin_gamma_statistics, pin_pack_words, pin_pack_exhaustive, pin_density, pin_act_ties,
     pin_act_amax_position, pin_act_symmetry_scaling, pin_brute_force, pin_addsub,
-    pin_ones_and_zero, pin_sign_flip, pin_epilogue, pin_bf16,
+    pin_ones_and_zero, pin_sign_flip, pin_epilogue, pin_bf16, pin_rms_norm,
 ]

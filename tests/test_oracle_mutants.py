@@ -35,6 +35,11 @@ MUTANTS = {
     "bf16_round_half_up": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0x8000u;"),
     "gamma_zero_guard_dropped": ("if (gamma == 0.0f)\n        return 0;\n    float t", "float t"),
     "ternary_threshold_shift": ("float t = w / gamma;", "float t = w / gamma * 0.9f;"),
+    "rms_norm_drops_eps": ("sqrt(ss / (double)K + 1e-6)", "sqrt(ss / (double)K)"),
+    "rms_norm_sum_not_mean": ("sqrt(ss / (double)K + 1e-6)", "sqrt(ss + 1e-6)"),
+    "rms_norm_no_sqrt": ("(float)(1.0 / sqrt(ss / (double)K + 1e-6))",
+                         "(float)(1.0 / (ss / (double)K + 1e-6))"),
+    "rms_norm_k_minus_one": ("sqrt(ss / (double)K + 1e-6)", "sqrt(ss / (double)(K - 1) + 1e-6)"),
 }
 
 
