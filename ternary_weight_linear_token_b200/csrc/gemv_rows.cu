@@ -322,8 +322,12 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       if (t >= p.M) break;
-      float a = 0.0f, inv = 1.0f;
-      for (int i = 0; i < nwarps; ++i) a = fmaxf(a, wmax[i * kMaxTok + t]);
+      // the per-warp maxima, one per lane, reduced by each warp at once (max
+      // is exact in any order; a loop over them cost every thread nwarps
+      // dependent shared-memory reads)
+      const float wm = lane < nwarps ? wmax[lane * kMaxTok + t] : 0.0f;
+      float a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(wm)));
+      float inv = 1.0f;
       if (NORM) {
         float ss = 0.0f;
         for (int i = 0; i < nwarps; ++i) ss = __fadd_rn(ss, wss[i * kMaxTok + t]);
