@@ -1,11 +1,20 @@
 """Benchmark of the B200 BitLinear forward (W1.58A8) -- one JSON line.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|chain]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload decode|prefill|sweep|chain] [--impl ours|reference]
 
 Metric: decode GEMV weight GB/s (packed 2-bit weight bytes streamed per
-second) and, for the prefill workload, int8 tensor-core TOPS (2*M*N*K per
-second), each against the B200 roofline.
+second) and prefill GEMM int8 TOPS (2*M*N*K per second), each against the
+B200 roofline.  The default run measures both: the decode GEMV is the line's
+own value, and the prefill GEMM (M=4096, K=2560, N=6912) its "prefill"
+object, each with its roofline, CPU oracle baseline, end-to-end figure and
+clocks.
+
+Every timed region is one replay of a CUDA graph of the K timed steps,
+bracketed by CUDA events on the launch stream; a spin kernel enqueued just
+before the first event keeps the GPU busy while the host submits the graph,
+so the events see the steps' device time and not the host's launch latency
+(the same number for --steps 20 as for --steps 2000).
 
 A step is one pass of the BitLinear forward over one batch of synthetic,
 seeded input: per-token activation quantisation, the ternary x int8
@@ -290,18 +299,30 @@ def make_prefill(tw, torch, dev, l2_bytes):
         tw.bitnet_w158a8_matmul(Xs[j], Ps[j], gamma, Y=Ys[j], workspace=wss[j],
                                 weights_static=True, stream=stream)
 
+    # The tensor-core kernel alone: int8 activations (natural K order) with
+    # their scales, and per set a workspace whose int8 weight copy a first,
+    # untimed call wrote; the timed calls promise that copy
+    # (weights_expanded), so each is exactly one tcgen05 kernel launch.
     qx = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(R)]
     qs = [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(R)]
+    need8 = tw.bitnet_w158a8_matmul_workspace_size(M, N, K, torch.int8)
+    ws8 = [torch.empty(need8, dtype=torch.uint8, device=dev) for _ in range(R)]
+    for j in range(R):
+        tw.bitnet_quantize_act(Xs[j], xq=qx[j], s=qs[j])
+        tw.bitnet_w158a8_matmul(qx[j], Ps[j], gamma, s=qs[j], Y=Ys[j], workspace=ws8[j])
 
-    def quant_step(i, stream=None):  # the step's activation quantiser alone
+    def kernel_step(i, stream=None):
         j = i % R
-        tw.bitnet_quantize_act(Xs[j], xq=qx[j], s=qs[j], stream=stream)
+        tw.bitnet_w158a8_matmul(qx[j], Ps[j], gamma, s=qs[j], Y=Ys[j], workspace=ws8[j],
+                                weights_static=True, weights_expanded=True, stream=stream)
 
     ops = 2 * M * N * K
     return dict(
-        step=step, kernel_step=None, quant_step=quant_step, units_per_step=ops, unit="TOPS",
+        step=step, kernel_step=kernel_step, e2e_step=lambda i, stream=None: step(0, stream),
+        units_per_step=ops, unit="TOPS",
         scale=1e-12,
-        bound="tensor", launches_per_step=2, rotate=R, X=X0, Y=Ys[0],
+        bound="tensor", launches_per_step=2, kernel_launches_per_step=1, rotate=R, X=X0,
+        Y=Ys[0], path=tw.bitnet_w158a8_matmul_path(M, N, K, torch.bfloat16),
         config={**workload_identity("prefill"),
                 "l2": f"inputs larger than L2: {R} rotating input/output sets",
                 "timing": "CUDA graph; step = activation quantiser (the weights' expansion to "
@@ -402,22 +423,29 @@ def oracle_sample(workload: str, budget_s: float, sweep_m: int = 8):
 
 
 # ------------------------------------------------------------------ main
+def oracle_run(workload: str, steps: int, warmup: int, per_step: float, sweep_m: int):
+    """The oracle timed over `steps` bounded samples of a workload (after
+    `warmup` shorter ones): (value, unit, cores, sample description, seconds)."""
+    for _ in range(warmup):
+        oracle_sample(workload, per_step / 4, sweep_m)
+    tot_units = 0.0
+    t0 = time.perf_counter()
+    cores, sample, unit = 1, "", "GB/s"
+    for _ in range(steps):
+        v, unit, cores, sample, dt = oracle_sample(workload, per_step, sweep_m)
+        tot_units += v * dt
+    dt = time.perf_counter() - t0
+    return tot_units / dt, unit, cores, sample, dt
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    per_step = max(0.02, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
-    for _ in range(args.warmup):
-        oracle_sample(args.workload, per_step / 4, args.sweep_m)
-    tot_units = 0.0
-    t0 = time.perf_counter()
-    cores = 1
-    sample = ""
-    unit = "GB/s"
-    for _ in range(args.steps):
-        v, unit, cores, sample, dt = oracle_sample(args.workload, per_step, args.sweep_m)
-        tot_units += v * dt
-    dt = time.perf_counter() - t0
-    value = tot_units / dt
+    with_prefill = args.workload == "decode" and not args.no_prefill
+    budget = 60.0 if with_prefill else 120.0
+    per_step = max(0.02, min(2.0, budget / max(1, args.steps + args.warmup)))
+    value, unit, cores, sample, dt = oracle_run(args.workload, args.steps, args.warmup, per_step,
+                                                args.sweep_m)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
@@ -428,8 +456,139 @@ def run_reference(args, world, rank):
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": f"per step ~{per_step:.2f} s of: {sample}"},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if with_prefill:
+        pv, pu, pc, ps, pdt = oracle_run("prefill", args.steps, args.warmup, per_step,
+                                         args.sweep_m)
+        line["prefill"] = {
+            "metric": "prefill GEMM int8 TOPS", "value": pv, "unit": pu,
+            "ms_per_step": 1e3 * pdt / max(1, args.steps),
+            "config": {**workload_identity("prefill"),
+                       "timing": "the oracle (plain C) on the host cores, a bounded sample of "
+                                 "the workload per step, scaled to the metric's unit"},
+            "cpu_baseline": {"value": pv, "unit": pu, "cores": pc, "kind": "oracle",
+                             "sample": f"per step ~{per_step:.2f} s of: {ps}"},
+            "e2e": {"value": pv, "unit": pu, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+# Spin cycles that keep the GPU busy while the host submits a timed graph:
+# the event pair then brackets the graph's device time alone, whatever the
+# host's launch latency (about 1 ms plus 1 us per graph node at ~2 GHz).
+def spin_cycles(nodes: int) -> int:
+    return int(2_000_000 + 2_000 * nodes)
+
+
+def capture(torch, stream, fn, first: int, count: int):
+    """One CUDA graph of `count` calls fn(first + i, stream)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(count):
+            fn(first + i, stream)
+    return g
+
+
+def replay_timed(torch, graph, stream, nodes: int, clocks=None):
+    """Device time (ms) of one replay of `graph`, CUDA events on `stream`.
+    A spin kernel ahead of the first event hides the host's graph submission."""
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(spin_cycles(nodes))
+        ev0.record(stream)
+        graph.replay()          # replays on the current stream, i.e. `stream`
+        ev1.record(stream)
+    ev1.synchronize()
+    return ev0.elapsed_time(ev1)
+
+
+def measure(w, tw, torch, args, dev, stream, pg, world, rank, bus):
+    """Warm-up, then the timed steps from one CUDA graph; the dominant
+    kernel's own time; end-to-end through the API; the oracle's CPU figure."""
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            w["step"](i, stream)
+    stream.synchronize()
+    graph = capture(torch, stream, w["step"], args.warmup, args.steps)
+    kgraph = None
+    if w.get("kernel_step") is not None and w["kernel_step"] is not w["step"]:
+        kgraph = capture(torch, stream, w["kernel_step"], 0, args.steps)
+    with torch.cuda.stream(stream):
+        graph.replay()  # one untimed replay of each: first-launch costs of the graphs
+        if kgraph is not None:
+            kgraph.replay()
+    stream.synchronize()
+
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    nodes = args.steps * w["launches_per_step"]
+    with ClockSampler(bus) as clocks:
+        ms = replay_timed(torch, graph, stream, nodes)
+        kms = ms
+        if kgraph is not None:
+            kms = replay_timed(torch, kgraph, stream, args.steps * w["kernel_launches_per_step"])
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    ms = max_over_ranks(ms, pg, dev)
+    kms = max_over_ranks(kms, pg, dev)
+    value = whole_job_value(world, w["units_per_step"], args.steps, ms * 1e-3, w["scale"])
+
+    per_launch_s = kms * 1e-3 / args.steps
+    pk, src = peaks()
+    if w["bound"] == "hbm":
+        peak, punit = float(pk["hbm_gbs"]), "GB/s"
+        achieved = w["units_per_step"] / per_launch_s * 1e-9
+        peak_note = f"hbm_gbs ({src}: STREAM-style copy)"
+    else:
+        peak, punit = float(pk["bf16_tflops"]) * INT8_PER_BF16, "TFLOP/s"
+        achieved = w["units_per_step"] / per_launch_s * 1e-12
+        peak_note = f"bf16_tflops x {INT8_PER_BF16} (int8/bf16 nominal ratio; {src} burst)"
+    traffic = ncu_traffic(w["kernel_key"], w["kernel_files"]) if w["kernel_key"] else None
+    roofline = {"bound": w["bound"], "achieved": achieved, "peak": peak, "unit": punit,
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
+                "kernel_us": 1e3 * kms / args.steps,
+                "kernel_timing": ("the tensor-core kernel alone: a CUDA graph of one launch "
+                                  "per step on prepared int8 activations and int8 weight "
+                                  "copies, CUDA events on the launch stream")
+                if kgraph is not None else "CUDA-event time of the timed steps"}
+
+    # end to end through the public API: pinned host input -> device -> result -> host
+    xh_np, h2d, d2h = w["e2e_inputs"]()
+    xh = torch.from_numpy(np.ascontiguousarray(xh_np)).pin_memory()
+    yh = torch.empty(w["Y"].shape, dtype=w["Y"].dtype).pin_memory()
+    X = w["X"]
+    e2e_step = w.get("e2e_step", w["step"])  # a step that reads X and writes Y
+    n = max(3, min(args.e2e_steps, args.steps))
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            X.view(torch.int16).copy_(xh.view(X.shape), non_blocking=True)
+            e2e_step(i, stream)
+            yh.copy_(w["Y"], non_blocking=True)
+        stream.synchronize()
+        t0 = time.perf_counter()
+        for i in range(n):
+            X.view(torch.int16).copy_(xh.view(X.shape), non_blocking=True)
+            e2e_step(i, stream)
+            yh.copy_(w["Y"], non_blocking=True)
+            stream.synchronize()
+        dt = time.perf_counter() - t0
+    dt = max_over_ranks(dt, pg, dev)
+    ev = whole_job_value(world, w["units_per_step"], n, dt, w["scale"])
+    e2e = {"value": ev, "unit": w["unit"], "h2d_bytes_per_step": int(h2d),
+           "d2h_bytes_per_step": int(d2h), "steps": n,
+           "note": "pinned host activations copied in, BitLinear via the Python binding of "
+                   "the C ABI, bf16 result copied out, stream synchronised, every step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        v, unit, cores, sample, cdt = oracle_sample(w["name"], args.cpu_seconds, args.sweep_m)
+        cpu = {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
+               "sample": f"{sample} in {cdt:.1f} s"}
+    del graph, kgraph
+    return dict(value=value, ms=ms, roofline=roofline, e2e=e2e, cpu_baseline=cpu,
+                clocks=clocks.summary(), gpu_launches=nodes)
 
 
 def main():
@@ -444,6 +603,8 @@ def main():
     ap.add_argument("--sweep-m", type=int, default=8, help="sweep workload: tokens per call")
     ap.add_argument("--chain-mode", choices=["persistent", "per-launch"], default="per-launch",
                     help="chain workload: one persistent kernel per token, or one launch per step")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode workload: leave out the prefill object of the JSON line")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world, rank, local = dist_setup()
@@ -466,132 +627,54 @@ def main():
         pg = dist
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2**20))
+    bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
+                                getattr(props, "pci_device_id", 0))
     extra = {"persistent": args.chain_mode == "persistent"} if args.workload == "chain" else {}
     if args.workload == "sweep":
         extra = {"M": args.sweep_m}
-    w = MAKERS[args.workload](tw, torch, dev, l2, **extra)
     stream = torch.cuda.Stream(dev)
+    w = MAKERS[args.workload](tw, torch, dev, l2, **extra)
+    w["name"] = args.workload
+    r = measure(w, tw, torch, args, dev, stream, pg, world, rank, bus)
+    cfg, unit = w["config"], w["unit"]
+    del w
 
-    # warm-up (eager launches), then capture the timed steps in one graph
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            w["step"](i, stream)
-    stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for i in range(args.steps):
-            w["step"](args.warmup + i, stream)
-    qgraph = None
-    if w.get("quant_step") is not None:
-        qgraph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(qgraph, stream=stream):
-            for i in range(args.steps):
-                w["quant_step"](i, stream)
-    with torch.cuda.stream(stream):
-        graph.replay()  # one untimed replay: first-launch costs of the graph
-    stream.synchronize()
-
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize(dev)
-    bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
-                                getattr(props, "pci_device_id", 0))
-    with ClockSampler(bus) as clocks, torch.cuda.stream(stream):
-        ev0.record(stream)
-        graph.replay()          # replays on the current stream, i.e. `stream`
-        ev1.record(stream)
-        ev1.synchronize()
-    torch.cuda.synchronize(dev)
-    if pg:
-        pg.barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
-    value = whole_job_value(world, w["units_per_step"], args.steps, ms * 1e-3, w["scale"])
-
-    # dominant kernel (prefill: the tcgen05 kernel = step minus its activation
-    # quantiser, each timed live with CUDA events on the same stream)
-    kms = ms
-    quant_ms = None
-    if qgraph is not None:
-        with torch.cuda.stream(stream):
-            qgraph.replay()
-            stream.synchronize()
-            ev0.record(stream)
-            qgraph.replay()
-            ev1.record(stream)
-            ev1.synchronize()
-        quant_ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
-        kms = ms - quant_ms
-    per_launch_s = kms * 1e-3 / args.steps
-    pk, src = peaks()
-    if w["bound"] == "hbm":
-        peak, punit = float(pk["hbm_gbs"]), "GB/s"
-        achieved = w["units_per_step"] / per_launch_s * 1e-9
-        peak_note = f"hbm_gbs ({src}: STREAM-style copy)"
-    else:
-        peak, punit = float(pk["bf16_tflops"]) * INT8_PER_BF16, "TFLOP/s"
-        achieved = w["units_per_step"] / per_launch_s * 1e-12
-        peak_note = f"bf16_tflops x {INT8_PER_BF16} (int8/bf16 nominal ratio; {src} burst)"
-    traffic = ncu_traffic(w["kernel_key"], w["kernel_files"]) if w["kernel_key"] else None
-
-    # end to end through the public API: pinned host input -> device -> result -> host
-    e2e = None
-    xh_np, h2d, d2h = w["e2e_inputs"]()
-    if True:
-        xh = torch.from_numpy(np.ascontiguousarray(xh_np)).pin_memory()
-        yh = torch.empty(w["Y"].shape, dtype=w["Y"].dtype).pin_memory()
-        X = w["X"]
-        n = max(3, min(args.e2e_steps, args.steps))
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                X.view(torch.int16).copy_(xh.view(X.shape), non_blocking=True)
-                w["step"](i, stream)
-                yh.copy_(w["Y"], non_blocking=True)
-            stream.synchronize()
-            t0 = time.perf_counter()
-            for i in range(n):
-                X.view(torch.int16).copy_(xh.view(X.shape), non_blocking=True)
-                w["step"](i, stream)
-                yh.copy_(w["Y"], non_blocking=True)
-                stream.synchronize()
-            dt = time.perf_counter() - t0
-        dt = max_over_ranks(dt, pg, dev)
-        ev = whole_job_value(world, w["units_per_step"], n, dt, w["scale"])
-        e2e = {"value": ev, "unit": w["unit"], "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": n,
-               "note": "pinned host activations copied in, BitLinear via the Python binding of "
-                       "the C ABI, bf16 result copied out, stream synchronised, every step"}
+    prefill = None
+    if args.workload == "decode" and not args.no_prefill:
+        # the other half of the metric: the prefill GEMM (M=4096, K=2560,
+        # N=6912) with the same timing rules, as its own object
+        wp = make_prefill(tw, torch, dev, l2)
+        wp["name"] = "prefill"
+        rp = measure(wp, tw, torch, args, dev, stream, pg, world, rank, bus)
+        prefill = {"metric": "prefill GEMM int8 TOPS", "value": rp["value"], "unit": "TOPS",
+                   "ms_per_step": rp["ms"] / args.steps,
+                   "config": dict(wp["config"], parallelism=f"replicas x{world}"
+                                  if world > 1 else "1 GPU"),
+                   "kernel_path": tw.PATH_NAMES.get(wp["path"], str(wp["path"])),
+                   "roofline": rp["roofline"], "cpu_baseline": rp["cpu_baseline"],
+                   "e2e": rp["e2e"], "clocks": rp["clocks"], "gpu_launches": rp["gpu_launches"]}
+        del wp
 
     status = tw.bitnet_get_device_status(stream)
-    cpu = None
-    if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        v, unit, cores, sample, dt = oracle_sample(args.workload, args.cpu_seconds, args.sweep_m)
-        cpu = {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
-               "sample": f"{sample} in {dt:.1f} s"}
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": w["unit"], "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "metric": METRIC, "value": r["value"], "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": r["ms"] / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
             "data": "synthetic (seeded; no dataset or trained weights)",
-            "config": dict(w["config"], parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
-            "roofline": {"bound": w["bound"], "achieved": achieved, "peak": peak, "unit": punit,
-                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
-                         "kernel_us": 1e3 * kms / args.steps,
-                         "kernel_timing": ("step time minus the time of the activation quantiser "
-                                           "alone (without the weight expansion, which the "
-                                           "kernel's figure therefore carries), both CUDA-event "
-                                           "timed on the launch stream")
-                         if quant_ms is not None else "CUDA-event time of the timed steps"},
-            "cpu_baseline": cpu,
-            "clocks": clocks.summary(),
-            "e2e": e2e,
-            "gpu_launches": w["launches_per_step"] * args.steps,
+            "config": dict(cfg,
+                           parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+            "roofline": r["roofline"],
+            "cpu_baseline": r["cpu_baseline"],
+            "clocks": r["clocks"],
+            "e2e": r["e2e"],
+            "gpu_launches": r["gpu_launches"],
             "device_status": int(status),
         }
+        if prefill is not None:
+            line["prefill"] = prefill
         print(json.dumps(line), flush=True)
-    del graph, qgraph
     if pg:
         pg.barrier()
         pg.destroy_process_group()

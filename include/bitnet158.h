@@ -93,6 +93,20 @@ typedef enum bitnet_epilogue {
  * weights are also read only after that point. */
 #define BITNET_FLAG_WEIGHTS_STATIC 1u
 
+/* Flag for bitnet_w158a8_matmul: the workspace already holds the int8 copy
+ * of these packed weights that the tensor-core path makes, written by an
+ * earlier call with the same `packed`, N, K and the same kind of input
+ * (int8 activations, or fp32/bf16 ones: the two keep the copy in different
+ * K orders), on this workspace, and nothing has written that part of the
+ * workspace since.  The call then skips the expansion and only quantises
+ * the activations (fp32/bf16 input) and runs the tensor-core kernel.  For a
+ * prefill that reuses one weight matrix over many calls (token blocks of a
+ * long prompt, several prompts in turn) this saves N*K/4 bytes read and N*K
+ * written per call.  Calls on the other paths keep no weight copy and
+ * ignore the flag (bitnet_w158a8_matmul_path tells which path a call
+ * takes).  A wrong promise gives wrong results, not an error. */
+#define BITNET_FLAG_WEIGHTS_EXPANDED 2u
+
 /* ----------------------------------------------------------------------
  * Weight quantisation: absmean ternary codes, packed four per byte.
  * ("Microsoft BitNet 深度研究报告", 技术原理 item 2; 2B4T report write-up,
@@ -143,7 +157,7 @@ bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M
  *   workspace at least bitnet_w158a8_matmul_workspace_size(M, N, K, x_dtype)
  *            bytes (may be NULL when that is 0).  Contents on entry don't
  *            matter; the call may overwrite all of it.
- *   flags    0 or BITNET_FLAG_WEIGHTS_STATIC.
+ *   flags    0, or BITNET_FLAG_WEIGHTS_STATIC and/or BITNET_FLAG_WEIGHTS_EXPANDED.
  * Up to 3 tokens (8 when K % 64 != 0) run one fused kernel and need no
  * workspace.  Otherwise fp32/bf16 input is first quantised into the
  * workspace by the activation quantiser (M*K bytes + 4*M, each rounded up to
@@ -160,6 +174,27 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                    int64_t N, int64_t K, bitnet_epilogue epi, void *Y,
                                    bitnet_dtype y_dtype, void *workspace, size_t workspace_bytes,
                                    uint32_t flags, bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
+ * Which kernel path bitnet_w158a8_matmul takes for these sizes on the
+ * current device (the paths are listed in the comment above).  Pure host
+ * logic, except that the tensor-core path also needs the driver's
+ * tensor-map encoder (cuTensorMapEncodeTiled), looked up once it is found:
+ * when the driver does not provide it, calls of the tensor-core shape run
+ * the much slower dp4a kernel instead, and this query returns
+ * BITNET_PATH_GENERIC for them, so that a caller can tell.  Returns
+ * BITNET_PATH_NONE for invalid sizes or dtypes, or an empty call.
+ * ---------------------------------------------------------------------- */
+typedef enum bitnet_path {
+    BITNET_PATH_NONE = 0,
+    BITNET_PATH_ROWS = 1,        /* 1..3 tokens (8 when K % 64 != 0): fused dp4a kernel        */
+    BITNET_PATH_MMA_TOKENS = 2,  /* 4..32 tokens, fp32/bf16 input: quantiser + int8 mma.sync  */
+    BITNET_PATH_MMA_WEIGHTS = 3, /* 9..32 tokens, int8 input: int8 mma.sync, weights as A     */
+    BITNET_PATH_TENSOR_CORE = 4, /* more tokens: weight expansion + tcgen05 kernel             */
+    BITNET_PATH_GENERIC = 5      /* K % 64 != 0, or no tensor-map encoder: dp4a fallback      */
+} bitnet_path;
+
+bitnet_path bitnet_w158a8_matmul_path(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype);
 
 /* ----------------------------------------------------------------------
  * Y = BitLinear(rms_norm(X)): the weightless RMS normalisation of
@@ -209,7 +244,10 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - All calls on a device share the one array, which keeps whatever the
- *     last call left in it; nothing in it needs to start at zero.  Calls
+ *     last call left in it; nothing in it needs to start at zero.
+ *     BITNET_FLAG_WEIGHTS_EXPANDED refers to that array here: it holds only
+ *     when the previous tensor-core-path call on the device used the same
+ *     weights and kind of input.  Calls
  *     whose kernels overlap on the GPU (different streams or threads) race
  *     on the array: keep them on one stream or otherwise serialised.
  * ---------------------------------------------------------------------- */

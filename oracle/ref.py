@@ -187,6 +187,37 @@ class COracle:
         return int(self.L.ref_num_threads())
 
 
+def decode_chain(x0, layers, d: int, oracle=None) -> list:
+    """A stack of decoder layers' BitLinear projections for one token, in
+    bf16 between projections (TEST INFRASTRUCTURE, composed of the functions
+    above only).  Per layer: q = BitLinear_qkv(x)[:, :d]; o = BitLinear_o(q);
+    u = ReLU^2(BitLinear_up(o)); v = BitLinear_down(u); x <- rms_norm(v).
+    (Model card of BitNet b1.58 2B4T, 模型详情 -> 架构: ReLU^2 in the FFN and a
+    "subln" normalisation without a formula; the weightless RMS
+    normalisation is the plain stand-in, and the first d columns of the QKV
+    output stand in for attention, which is not part of the path.)
+
+    x0: fp32 [1, K] (bf16-exact values); layers: per layer four
+    (packed, gamma, N, relu2).  Returns per layer the bf16 bit patterns of
+    [qkv, o, up, down, normalised] outputs."""
+    R = oracle or default()
+    x = np.ascontiguousarray(x0, dtype=np.float32)
+    outs = []
+    for proj in layers:
+        bits = []
+        inp = x
+        for pi, (packed, gamma, N, relu2) in enumerate(proj):
+            y = R.to_bf16(R.bitlinear(inp, packed, gamma, N, relu2=relu2)["y"])
+            bits.append(y)
+            f = (y.astype(np.uint32) << 16).view(np.float32)
+            inp = f[:, :d] if pi == 0 else f
+        n = R.to_bf16(R.rms_norm(inp))
+        bits.append(n)
+        x = (n.astype(np.uint32) << 16).view(np.float32)
+        outs.append(bits)
+    return outs
+
+
 _default = None
 
 

@@ -32,6 +32,11 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOU
 F32, BF16, I8, I32 = 0, 1, 2, 3
 EPI_NONE, EPI_RELU2 = 0, 1
 FLAG_WEIGHTS_STATIC = 1
+FLAG_WEIGHTS_EXPANDED = 2
+PATH_NONE, PATH_ROWS, PATH_MMA_TOKENS, PATH_MMA_WEIGHTS, PATH_TENSOR_CORE, PATH_GENERIC = range(6)
+PATH_NAMES = {PATH_NONE: "none", PATH_ROWS: "rows", PATH_MMA_TOKENS: "mma_tokens",
+              PATH_MMA_WEIGHTS: "mma_weights", PATH_TENSOR_CORE: "tensor_core",
+              PATH_GENERIC: "generic"}
 
 _DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.int8: I8, torch.int32: I32}
 
@@ -48,6 +53,7 @@ _SIGS = {
     "bitnet_quantize_weights": ([_P, _ST, _I64, _I64, _P, _P, _P, _SZ, _P], _ST),
     "bitnet_quantize_act": ([_P, _ST, _I64, _I64, _P, _P, _P], _ST),
     "bitnet_w158a8_matmul_workspace_size": ([_I64, _I64, _I64, _ST], _SZ),
+    "bitnet_w158a8_matmul_path": ([_I64, _I64, _I64, _ST], _ST),
     "bitnet_w158a8_matmul": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST, _P, _SZ,
                               C.c_uint32, _P], _ST),
     "bitnet_rms_norm": ([_P, _ST, _I64, _I64, _P, _ST, _P], _ST),
@@ -169,14 +175,23 @@ def bitnet_w158a8_matmul_workspace_size(M: int, N: int, K: int, x_dtype) -> int:
     return lib.bitnet_w158a8_matmul_workspace_size(M, N, K, xd)
 
 
+def bitnet_w158a8_matmul_path(M: int, N: int, K: int, x_dtype) -> int:
+    """The kernel path a call of these sizes takes on the current device
+    (one of the PATH_* constants)."""
+    xd = _DTYPE[x_dtype] if isinstance(x_dtype, torch.dtype) else int(x_dtype)
+    return lib.bitnet_w158a8_matmul_path(M, N, K, xd)
+
+
 def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
                          s: torch.Tensor | None = None, relu2: bool = False,
                          out_dtype: torch.dtype = torch.bfloat16, Y: torch.Tensor | None = None,
                          workspace: torch.Tensor | None = None, weights_static: bool = False,
-                         stream=None) -> torch.Tensor:
+                         weights_expanded: bool = False, stream=None) -> torch.Tensor:
     """Y = BitLinear(X).  X is fp32/bf16 [M, K] (quantised inside the call) or
     int8 xq [M, K] with its scales ``s`` [M].  out_dtype fp32/bf16, or int32
-    for the raw accumulators (relu2 must then be False)."""
+    for the raw accumulators (relu2 must then be False).  ``weights_expanded``
+    promises that ``workspace`` still holds the int8 weight copy of an
+    earlier tensor-core-path call with the same weights and input kind."""
     _dev(X, "X", (torch.float32, torch.bfloat16, torch.int8))
     _dev(packed, "packed", (torch.uint8,))
     _dev(gamma, "gamma", (torch.float32,))
@@ -196,7 +211,9 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
     st = lib.bitnet_w158a8_matmul(_ptr(X), _DTYPE[X.dtype], _ptr(s), _ptr(packed), _ptr(gamma),
                                   M, N, K, EPI_RELU2 if relu2 else EPI_NONE, _ptr(Y),
                                   _DTYPE[Y.dtype], _ptr(workspace), ws_bytes,
-                                  FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
+                                  (FLAG_WEIGHTS_STATIC if weights_static else 0)
+                                  | (FLAG_WEIGHTS_EXPANDED if weights_expanded else 0),
+                                  _stream(stream))
     _check(st, "bitnet_w158a8_matmul")
     return Y
 

@@ -33,21 +33,28 @@ from . import (bitnet_decode_chain, bitnet_decode_chain_steps, bitnet_decode_cha
 
 class DecodeChain:
     def __init__(self, weights, device="cuda:0", weights_static: bool = True,
-                 persistent: bool = False):
+                 persistent: bool = False, quantized=None):
         """weights: list over layers of a list of 4 (W [N, K] float tensor,
-        relu2) pairs in the order qkv, o, up, down.  Weights are quantised on
-        the device once, here."""
+        relu2) pairs in the order qkv, o, up, down (any iterable: a
+        generator keeps only one layer's latent weights alive at a time).
+        Weights are quantised on the device once, here.
+        quantized: instead of weights, the ``layers`` of another DecodeChain
+        (packed weights shared, nothing quantised again)."""
         self.device = torch.device(device)
         self.weights_static = weights_static
-        self.layers = []
-        for layer in weights:
-            proj = []
-            for W, relu2 in layer:
-                W = W.to(self.device).contiguous()
-                packed, gamma = bitnet_quantize_weights(W)
-                proj.append(dict(packed=packed, gamma=gamma, N=W.shape[0], K=W.shape[1],
-                                 relu2=relu2))
-            self.layers.append(proj)
+        if quantized is not None:
+            self.layers = quantized
+        else:
+            self.layers = []
+            for layer in weights:
+                proj = []
+                for W, relu2 in layer:
+                    W = W.to(self.device).contiguous()
+                    packed, gamma = bitnet_quantize_weights(W)
+                    proj.append(dict(packed=packed, gamma=gamma, N=W.shape[0], K=W.shape[1],
+                                     relu2=relu2))
+                    del W
+                self.layers.append(proj)
         d = self.layers[0][1]["K"]
         self.d = d
         # activation buffers, one per step, kept so every link can be checked

@@ -135,14 +135,15 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                            const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
                            int64_t K, bitnet_epilogue epi, const void *Y, bitnet_dtype y_dtype,
                            const void *workspace, size_t workspace_bytes, uint32_t flags,
-                           bool norm_in) {
+                           bool norm_in, bool check_workspace = true) {
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
     return BITNET_ERR_INVALID_ARG;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32)
     return BITNET_ERR_INVALID_ARG;
   if (epi != BITNET_EPI_NONE && epi != BITNET_EPI_RELU2) return BITNET_ERR_INVALID_ARG;
   if (y_dtype == BITNET_I32 && epi != BITNET_EPI_NONE) return BITNET_ERR_INVALID_ARG;
-  if ((flags & ~BITNET_FLAG_WEIGHTS_STATIC) != 0) return BITNET_ERR_INVALID_ARG;
+  if ((flags & ~(BITNET_FLAG_WEIGHTS_STATIC | BITNET_FLAG_WEIGHTS_EXPANDED)) != 0)
+    return BITNET_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
   if (bitnet_status st = check_k(K)) return st;
   if (M == 0 || N == 0) return BITNET_OK;
@@ -156,6 +157,7 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
               static_cast<size_t>(M) * N * elem_size(y_dtype)))
     return BITNET_ERR_INVALID_ARG;
   // the normalising variant runs the fused kernel, with no scratch, whenever it can
+  if (!check_workspace) return BITNET_OK;
   const size_t need = norm_in && rows_supported(M, N, K) ? 0 : matmul_workspace(M, N, K, x_dtype);
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need) return BITNET_ERR_WORKSPACE;
@@ -169,7 +171,7 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
 bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                          const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
                          int64_t K, bool relu2, void *Y, bitnet_dtype y_dtype, void *workspace,
-                         bool wstatic, const LaunchCtx &ctx) {
+                         bool wstatic, bool expanded, const LaunchCtx &ctx) {
   if (use_rows(M, N, K, x_dtype))
     return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                  wstatic, false, nullptr, ctx));
@@ -183,7 +185,7 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
   if (prefill) {
     expand.packed = packed;
     expand.w8 = static_cast<int8_t *>(workspace) + (from_float ? act_scratch(M, K) : 0);
-    expand.words = N * (K / 16);
+    expand.words = expanded ? 0 : N * (K / 16);  // the caller vouches for an earlier expansion
   }
   if (from_float) {
     // The prefill and mmv kernels take the quantiser's output in the K order
@@ -196,7 +198,7 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     xq = wxq;
     sq = ws;
-  } else if (prefill) {
+  } else if (prefill && expand.words > 0) {
     // the caller's int8 activations are in natural K order
     if (launch_expand_weights(expand, false, ctx) != cudaSuccess) return BITNET_ERR_CUDA;
   }
@@ -241,6 +243,17 @@ size_t chain_workspace(const bitnet_chain_step *steps, int n_steps) {
 }
 
 }  // namespace
+
+// The argument checks of bitnet_w158a8_matmul without the workspace ones
+// (for the entry point that brings its own scratch).
+int matmul_args_status(const void *X, int x_dtype, const float *s, const uint8_t *packed,
+                       const float *gamma, int64_t M, int64_t N, int64_t K, int epi,
+                       const void *Y, int y_dtype, uint32_t flags) {
+  return check_matmul(X, static_cast<bitnet_dtype>(x_dtype), s, packed, gamma, M, N, K,
+                      static_cast<bitnet_epilogue>(epi), Y, static_cast<bitnet_dtype>(y_dtype),
+                      nullptr, 0, flags, false, false);
+}
+
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -307,6 +320,19 @@ size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitn
   return matmul_workspace(M, N, K, x_dtype);
 }
 
+bitnet_path bitnet_w158a8_matmul_path(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
+    return BITNET_PATH_NONE;
+  if (M <= 0 || N <= 0 || M > kMaxRows || N > kMaxRows || check_k(K) != BITNET_OK)
+    return BITNET_PATH_NONE;
+  if (use_rows(M, N, K, x_dtype)) return BITNET_PATH_ROWS;
+  if (x_dtype != BITNET_I8 && mmv_supported(M, N, K)) return BITNET_PATH_MMA_TOKENS;
+  if (x_dtype == BITNET_I8 && decode_supported(M, N, K)) return BITNET_PATH_MMA_WEIGHTS;
+  // the same decision run_matmul takes, the encoder lookup included
+  if (use_prefill(M, N, K, x_dtype) && prefill_supported(M, N, K)) return BITNET_PATH_TENSOR_CORE;
+  return BITNET_PATH_GENERIC;
+}
+
 bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                                    const uint8_t *packed, const float *gamma, int64_t M,
                                    int64_t N, int64_t K, bitnet_epilogue epi, void *Y,
@@ -319,7 +345,8 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
   LaunchCtx ctx;
   if (bitnet_status st = device_ctx(stream, &ctx)) return st;
   return run_matmul(X, x_dtype, s, packed, gamma, M, N, K, epi == BITNET_EPI_RELU2, Y, y_dtype,
-                    workspace, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0, ctx);
+                    workspace, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0,
+                    (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0, ctx);
 }
 
 bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype, void *X_normed,
@@ -351,7 +378,7 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
                                  wstatic, true, X_normed, ctx));
   if (launch_rms_norm(X, x_dtype, M, K, X_normed, x_dtype, ctx) != cudaSuccess) return BITNET_ERR_CUDA;
   return run_matmul(X_normed, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                    workspace, wstatic, ctx);
+                    workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0, ctx);
 }
 
 bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K, void *Y,

@@ -290,6 +290,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 
 // ------------------------------------------------------------ arithmetic
 // Per-token scale s = 127 / amax (IEEE fp32 division); 1 for an all-zero row.
+// The weightless RMS normalisation's factor 1 / sqrt(ss / K + 1e-6) for a
+// token whose squares sum to ss.  ss is accumulated in fp64, where the square
+// of an fp32 (or bf16) value is exact, and the factor is computed in fp64 and
+// rounded once to fp32: the operations of the plain definition, so the
+// factor differs from it only where the fp64 sums, taken in another order,
+// straddle an fp32 rounding boundary of the factor (about one token in 10^7).
+__device__ __forceinline__ float rms_factor(double ss, int64_t K) {
+  const double q = __dadd_rn(__ddiv_rn(ss, static_cast<double>(K)), 1e-6);
+  return __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(q)));
+}
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+// x^2 added to an fp64 sum (the product is exact in fp64).
+__device__ __forceinline__ double add_sq(double ss, float x) {
+  const double d = static_cast<double>(x);
+  return __fma_rn(d, d, ss);
+}
+
 __device__ __forceinline__ float act_scale(float amax) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(127.0f, amax);
 }

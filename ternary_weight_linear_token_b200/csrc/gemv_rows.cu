@@ -59,9 +59,9 @@ struct RowsParams {
   int rpw;       // rows per warp in the dot products (1, 2 or 4; > 1 only for M <= 2)
 };
 
-// scales [kMaxTok], gamma/s [kMaxTok], then per-warp maxima and sums of
-// squares [kMaxWarps][kMaxTok] each
-constexpr int kHeader = 32 + 32 + 2 * kMaxWarps * kMaxTok * 4;
+// scales [kMaxTok], gamma/s [kMaxTok], per-warp maxima [kMaxWarps][kMaxTok]
+// (fp32), then per-warp sums of squares [kMaxWarps][kMaxTok] (fp64)
+constexpr int kHeader = 32 + 32 + kMaxWarps * kMaxTok * 4 + kMaxWarps * kMaxTok * 8;
 int x_row_bytes(int K) { return (K + 127) / 128 * 128; }
 int w_row_bytes(int K) { return (K / 4 + 15) / 16 * 16; }
 // One CTA per SM, so that a wide projection never runs a second wave (two
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
   float *s_sh = reinterpret_cast<float *>(smem);                 // kMaxTok scales
   float *r_sh = reinterpret_cast<float *>(smem + 32);            // kMaxTok gamma / s
   float *wmax = reinterpret_cast<float *>(smem + 64);            // [kMaxWarps][kMaxTok]
-  float *wss = wmax + kMaxWarps * kMaxTok;                       // [kMaxWarps][kMaxTok]
+  double *wss = reinterpret_cast<double *>(wmax + kMaxWarps * kMaxTok);  // [kMaxWarps][kMaxTok]
   uint8_t *xsh = smem + kHeader;
   uint8_t *wsh = xsh + p.M * p.xs;  // the host sizes shared memory for p.M token rows
 
@@ -251,10 +251,19 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
   const int rows = n1 - n0;
   const int words = p.K / 16;
 
-  if (p.weights_static) start_weight_copy(p, n0, rows, wsh);
+  // gamma belongs to the weights: with static weights it is read before the
+  // wait too, so its load is not on the path from the wait to the epilogue
+  float gamma = 0.0f;
+  if (p.weights_static) {
+    start_weight_copy(p, n0, rows, wsh);
+    gamma = *p.gamma;
+  }
   pdl_launch_dependents();
   pdl_wait();
-  if (!p.weights_static) start_weight_copy(p, n0, rows, wsh);
+  if (!p.weights_static) {
+    start_weight_copy(p, n0, rows, wsh);
+    gamma = *p.gamma;
+  }
 
   // ---- activations -> shared memory (int8, unpack order), per-token scales
   if (XK == kI8) {
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
     }
     if (tid < p.M) {
       s_sh[tid] = p.s_in[tid];
-      r_sh[tid] = __fdiv_rn(*p.gamma, p.s_in[tid]);
+      r_sh[tid] = __fdiv_rn(gamma, p.s_in[tid]);
     }
   } else {
     const int chunks = p.K / 8;
@@ -286,7 +295,8 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       if (t >= p.M) break;
-      float a = 0.0f, ss = 0.0f;
+      float a = 0.0f;
+      double ss = 0.0;
       if (tid < chunks) {
         float v[8];
         if (t < kCached)
@@ -296,7 +306,7 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           a = fmaxf(a, fabsf(v[e]));
-          if (NORM) ss = __fmaf_rn(v[e], v[e], ss);
+          if (NORM) ss = add_sq(ss, v[e]);
         }
       }
       for (int c = tid + blockDim.x; c < chunks; c += blockDim.x) {
@@ -305,14 +315,11 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           a = fmaxf(a, fabsf(v[e]));
-          if (NORM) ss = __fmaf_rn(v[e], v[e], ss);
+          if (NORM) ss = add_sq(ss, v[e]);
         }
       }
       a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
-      if (NORM) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
-      }
+      if (NORM) ss = warp_sum_f64(ss);
       if (lane == 0) {
         wmax[warp * kMaxTok + t] = a;
         if (NORM) wss[warp * kMaxTok + t] = ss;
@@ -329,9 +336,8 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
       float a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(wm)));
       float inv = 1.0f;
       if (NORM) {
-        float ss = 0.0f;
-        for (int i = 0; i < nwarps; ++i) ss = __fadd_rn(ss, wss[i * kMaxTok + t]);
-        inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, static_cast<float>(p.K)), 1e-6f)));
+        // the per-warp sums, one per lane, summed by each warp at once (fp64)
+        inv = rms_factor(warp_sum_f64(lane < nwarps ? wss[lane * kMaxTok + t] : 0.0), p.K);
         // rounding x * inv to the input's precision is monotone in |x|: the
         // max of the normalised values is the normalised max
         a = round_to_input<XK>(__fmul_rn(a, inv));
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(32 * warp_cap<MT>(), 1) rows_kernel(const Rows
       const bool write_n = NORM && p.Xn != nullptr && blockIdx.x == 0;
       if (tid == blockDim.x - 1) {  // a lane with no activation work in the common case
         s_sh[t] = sm;
-        r_sh[t] = __fdiv_rn(*p.gamma, sm);
+        r_sh[t] = __fdiv_rn(gamma, sm);
       }
       uint8_t *xrow = xsh + t * p.xs;
       {

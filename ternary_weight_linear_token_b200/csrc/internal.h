@@ -114,6 +114,12 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
                          const void *x0, void *y_norm, int64_t y_norm_n, void *workspace,
                          const LaunchCtx &ctx);
 
+// abi.cu: the argument checks of bitnet_w158a8_matmul without the workspace
+// ones, as a bitnet_status value (0 = OK).
+int matmul_args_status(const void *X, int x_dtype, const float *s, const uint8_t *packed,
+                       const float *gamma, int64_t M, int64_t N, int64_t K, int epi,
+                       const void *Y, int y_dtype, uint32_t flags);
+
 // Launch helper: cudaLaunchKernelEx with the PDL attribute when ctx.pdl.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,

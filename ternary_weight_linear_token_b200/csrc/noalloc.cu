@@ -55,9 +55,13 @@ extern "C" bitnet_status bitnet_w158a8_matmul_noalloc(const void *X, bitnet_dtyp
                                                       int64_t K, bitnet_epilogue epi, void *Y,
                                                       bitnet_dtype y_dtype, uint32_t flags,
                                                       bitnet_stream_t stream) {
-  // Size limit first, so an oversized call fails with the workspace status
-  // before anything touches the device.
-  if (M > 0 && N > 0 && K > 0 &&
+  // The regular argument checks first (a bad dtype, flag or size is an
+  // invalid argument, whatever scratch it would need), then the size limit;
+  // both before anything touches the device.
+  if (const int st = bitnet::matmul_args_status(X, x_dtype, s, packed, gamma, M, N, K, epi, Y,
+                                                y_dtype, flags))
+    return static_cast<bitnet_status>(st);
+  if (M > 0 && N > 0 &&
       bitnet_w158a8_matmul_workspace_size(M, N, K, x_dtype) > BITNET_STATIC_SCRATCH_BYTES)
     return BITNET_ERR_WORKSPACE;
   void *scratch = nullptr;

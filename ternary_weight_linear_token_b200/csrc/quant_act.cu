@@ -57,11 +57,6 @@ __device__ __forceinline__ float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 constexpr int kExpandWords = 4;  // packed words per thread
 constexpr int64_t kExpandBlockWords = 32 * kRowsPerCta * kExpandWords;
@@ -345,16 +340,14 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) rms_norm_kernel(const void *
   const int64_t m = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + (threadIdx.x >> 5);
   if (m < M) {
     const int64_t chunks = K / 16;
-    float ss = 0.0f;
+    double ss = 0.0;
     for (int64_t c = lane; c < chunks; c += 32) {
       float v[16];
       load16<XK>(X, m * K + 16 * c, v);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) ss = __fmaf_rn(v[e], v[e], ss);
+      for (int e = 0; e < 16; ++e) ss = add_sq(ss, v[e]);
     }
-    ss = warp_sum(ss);
-    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, static_cast<float>(K)),
-                                                           1e-6f)));
+    const float inv = rms_factor(warp_sum_f64(ss), K);
     for (int64_t c = lane; c < chunks; c += 32) {
       float v[16];
       load16<XK>(X, m * K + 16 * c, v);

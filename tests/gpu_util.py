@@ -53,6 +53,20 @@ def assert_f32_close(got: np.ndarray, want: np.ndarray, rel: float = 1e-6):
                            f"first at {np.argwhere(bad)[0]}: got {got[bad][0]!r} want {want[bad][0]!r}")
 
 
+def assert_f32_within_ulp(got: np.ndarray, want: np.ndarray, ulps: int):
+    """fp32 outputs: at most `ulps` units in the last place apart."""
+    g = np.asarray(got, dtype=np.float32).view(np.int32).astype(np.int64)
+    w = np.asarray(want, dtype=np.float32).view(np.int32).astype(np.int64)
+    assert g.shape == w.shape
+
+    def ordered(b):  # monotone integer image of the fp32 value line
+        return np.where(b < 0, -(b & 0x7FFFFFFF), b)
+    diff = np.abs(ordered(g) - ordered(w))
+    bad = diff > ulps
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} fp32 outputs more than {ulps} ulp apart; "
+                           f"first at {np.argwhere(bad)[0]}")
+
+
 def assert_bf16_within_ulp(got_bits: np.ndarray, want_bits: np.ndarray, ulps: int = 1):
     """bf16 outputs: at most `ulps` units in the last place apart (same sign
     or both zero)."""

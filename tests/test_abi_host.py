@@ -70,7 +70,7 @@ def test_matmul_rejects_bad_arguments(tw):
     assert mm(tw, yd=2) == tw.ERR_INVALID_ARG            # int8 output
     assert mm(tw, epi=2) == tw.ERR_INVALID_ARG
     assert mm(tw, yd=3, epi=1) == tw.ERR_INVALID_ARG     # raw int32 with ReLU^2
-    assert mm(tw, flags=2) == tw.ERR_INVALID_ARG
+    assert mm(tw, flags=4) == tw.ERR_INVALID_ARG         # unknown flag bit
     assert mm(tw, M=-1) == tw.ERR_INVALID_ARG
     assert mm(tw, K=0) == tw.ERR_INVALID_ARG
     assert mm(tw, K=40) == tw.ERR_UNSUPPORTED_SHAPE      # not a multiple of 16
@@ -198,4 +198,47 @@ def test_rms_norm_matmul_rejects_bad_arguments(tw):
     assert call(Xn=MIS) == tw.ERR_MISALIGNED
     assert call(Xn=C.c_void_p(0x10000000)) == tw.ERR_INVALID_ARG  # X_normed overlapping X
     assert call(Xn=C.c_void_p(0x30000000)) == tw.ERR_INVALID_ARG  # X_normed overlapping Y
+    assert call(M=0) == tw.OK
+
+
+def test_matmul_path_query(tw):
+    """Which kernel path a call takes: host logic for every path; the
+    tensor-core path also needs the driver's tensor-map encoder, which this
+    GPU-less host lacks, so calls of that shape report the dp4a fallback
+    instead of running it silently."""
+    f = tw.lib.bitnet_w158a8_matmul_path
+    assert f(1, 2560, 2560, tw.BF16) == tw.PATH_ROWS
+    assert f(3, 6912, 2560, tw.F32) == tw.PATH_ROWS
+    assert f(8, 2560, 2560, tw.BF16) == tw.PATH_MMA_TOKENS
+    assert f(32, 2560, 6912, tw.BF16) == tw.PATH_MMA_TOKENS
+    assert f(16, 2560, 2560, tw.I8) == tw.PATH_MMA_WEIGHTS
+    assert f(8, 2560, 2560, tw.I8) == tw.PATH_ROWS        # caller's int8, up to 8 tokens
+    assert f(5, 64, 48, tw.F32) == tw.PATH_ROWS           # K % 64 != 0, M <= 8
+    assert f(9, 64, 48, tw.F32) == tw.PATH_GENERIC        # K % 64 != 0, M > 8
+    assert f(0, 64, 64, tw.F32) == tw.PATH_NONE
+    assert f(4, 64, 40, tw.F32) == tw.PATH_NONE
+    assert f(4, 64, 64, 3) == tw.PATH_NONE                # int32 activations
+    import torch
+    want = tw.PATH_TENSOR_CORE if torch.cuda.is_available() else tw.PATH_GENERIC
+    assert f(4096, 6912, 2560, tw.BF16) == want
+    assert f(4096, 6912, 2560, tw.I8) == want
+
+
+def test_noalloc_checks_arguments_before_its_size_limit(tw):
+    """A bad dtype, flag or size is an invalid argument, even where the call
+    would also need more than the built-in scratch array; the size limit is
+    checked next; nothing reaches the device."""
+    f = tw.lib.bitnet_w158a8_matmul_noalloc
+
+    def call(X=A, xd=1, s=None, M=4096, N=6912, K=2560, epi=0, Y=Cc, yd=1, flags=0):
+        return f(X, xd, s, B, G, M, N, K, epi, Y, yd, flags, None)
+
+    assert call(xd=3) == tw.ERR_INVALID_ARG
+    assert call(xd=7) == tw.ERR_INVALID_ARG
+    assert call(yd=2) == tw.ERR_INVALID_ARG
+    assert call(flags=8) == tw.ERR_INVALID_ARG
+    assert call(M=1 << 40) == tw.ERR_INVALID_ARG
+    assert call(K=40) == tw.ERR_UNSUPPORTED_SHAPE
+    assert call(X=MIS) == tw.ERR_MISALIGNED
+    assert call(M=8192) == tw.ERR_WORKSPACE               # (8192 + 6912) * 2560 > 32 MiB
     assert call(M=0) == tw.OK

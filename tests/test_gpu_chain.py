@@ -177,3 +177,118 @@ def test_decode_chain_bounded_wait_reports_timeout(tw):
     check_links(steps, Ws, x0)
     assert int(ws.view(torch.int32)[0].item()) == 0  # launch counter unchanged
     assert tw.bitnet_get_device_status() == tw.OK   # reading the status cleared it
+
+
+# ------------------------------------------------------------------ the 30-layer stack
+@pytest.fixture(scope="module")
+def stack30(tw):
+    """The configured 30-layer decode stack (per layer qkv 2560->3840, o
+    2560->2560, up 2560->6912 + ReLU^2, down 6912->2560; 1.55 B ternary
+    weights): latent weights made one layer at a time, quantised on the GPU
+    and by the oracle (codes and gamma must agree), and both chain forms
+    sharing the GPU's packed weights.  Also the oracle's own run of the whole
+    stack from the chain input."""
+    from ternary_weight_linear_token_b200.chain import DecodeChain
+    layers = 30
+    oracle_layers = []
+
+    def gen():
+        for li in range(layers):
+            dev_w, proj = [], []
+            for p in range(4):
+                W = synth.layer_weights(li, p)
+                po, go = ref.quantize_weights(W)
+                proj.append((po, go, W.shape[0], synth.PROJECTIONS[p][3]))
+                dev_w.append((f32_t(W), synth.PROJECTIONS[p][3]))
+            oracle_layers.append(proj)
+            yield dev_w
+
+    per = DecodeChain(gen())
+    for li in range(layers):
+        for p in range(4):
+            po, go = oracle_layers[li][p][:2]
+            assert np.array_equal(np_of(per.layers[li][p]["packed"]), po), (li, p)
+            assert np_of(per.layers[li][p]["gamma"])[0] == go, (li, p)
+    pers = DecodeChain(None, persistent=True, quantized=per.layers)
+    x0 = synth.config_inputs("chain", weights=False)
+    want = ref.decode_chain(x0["x"], oracle_layers, per.d)
+    return dict(per=per, pers=pers, oracle=oracle_layers, x0=x0, want=want)
+
+
+def check_stack(chain, oracle_layers, x0_bits):
+    """Every link of a chain run: each projection's bf16 output bit-exact
+    against the oracle's BitLinear of the projection's actual bf16 input;
+    each normalised vector within 1 bf16 ulp of the oracle's normalisation
+    of the actual down output.  Returns how many normalised vectors are
+    bit-identical to the oracle's."""
+    d = chain.d
+    x_in = x0_bits.reshape(1, -1)
+    exact_norms = 0
+    for li, bufs in enumerate(chain.outs):
+        inputs = [x_in, bf16_bits_of(bufs[0])[:, :d], bf16_bits_of(bufs[1]), bf16_bits_of(bufs[2])]
+        for pi in range(4):
+            po, go, N, relu2 = oracle_layers[li][pi]
+            xin = synth.bf16_bits_to_f32(inputs[pi])
+            want = ref.to_bf16(ref.bitlinear(xin, po, go, N, relu2=relu2)["y"])
+            got = bf16_bits_of(bufs[pi])
+            bad = np.flatnonzero(got != want)
+            assert bad.size == 0, (li, pi, bad[:4], got.ravel()[bad[:4]], want.ravel()[bad[:4]])
+        want_n = ref.to_bf16(ref.rms_norm(synth.bf16_bits_to_f32(bf16_bits_of(bufs[3]))))
+        got_n = bf16_bits_of(bufs[4])
+        assert_bf16_within_ulp(got_n, want_n, 1)
+        exact_norms += int(np.array_equal(got_n, want_n))
+        x_in = got_n
+    return exact_norms
+
+
+def test_stack30_per_launch_links_and_end_to_end(tw, stack30):
+    """The per-launch form (121 launches per token) of the 30-layer stack:
+    all 120 BitLinear links and 30 normalisations against the oracle, then
+    the whole run against the oracle's own run from the chain input.  The
+    normalisation computes the oracle's fp64 sum and factor, so it is
+    bit-identical except where two fp64 summation orders straddle an fp32
+    rounding boundary of the factor (about 1e-7 per token); with every link
+    exact the whole stack then equals the oracle's run bit for bit.  Then a
+    CUDA-graph replay of the whole token reproduces the eager run."""
+    chain, x0 = stack30["per"], stack30["x0"]
+    chain.run(bf16_t(x0["x_bits"]).view(1, -1))
+    torch.cuda.synchronize()
+    exact = check_stack(chain, stack30["oracle"], x0["x_bits"])
+    assert exact >= 29, exact
+    if exact == 30:
+        for li, (bufs, want) in enumerate(zip(chain.outs, stack30["want"])):
+            for pi in range(5):
+                assert np.array_equal(bf16_bits_of(bufs[pi]), want[pi]), (li, pi)
+    eager = [bf16_bits_of(b).copy() for bufs in chain.outs for b in bufs]
+    for bufs in chain.outs:
+        for b in bufs:
+            b.fill_(float("nan"))
+    chain.capture()
+    chain.graph.replay()
+    torch.cuda.synchronize()
+    again = [bf16_bits_of(b) for bufs in chain.outs for b in bufs]
+    assert all(np.array_equal(a, b) for a, b in zip(eager, again))
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
+def test_stack30_persistent_links(tw, stack30):
+    """The persistent form (one bitnet_decode_chain launch per token, 120
+    steps, the 8-slot weight ring wrapping 15 times) of the 30-layer stack:
+    every link against the oracle, on two launches in a row (the second
+    with another input) and on a CUDA-graph replay."""
+    chain, x0 = stack30["pers"], stack30["x0"]
+    for r in range(2):
+        bits = x0["x_bits"] if r == 0 else x0_bits(2560, 77)
+        chain.run(bf16_t(bits).view(1, -1))
+        torch.cuda.synchronize()
+        check_stack(chain, stack30["oracle"], bits)
+    eager = [bf16_bits_of(b).copy() for bufs in chain.outs for b in bufs]
+    chain.capture()
+    for bufs in chain.outs:
+        for b in bufs:
+            b.fill_(float("nan"))
+    chain.graph.replay()
+    torch.cuda.synchronize()
+    assert all(np.array_equal(a, bf16_bits_of(b)) for a, b in
+               zip(eager, [b for bufs in chain.outs for b in bufs]))
+    assert tw.bitnet_get_device_status() == tw.OK
