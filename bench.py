@@ -10,11 +10,14 @@ own value, and the prefill GEMM (M=4096, K=2560, N=6912) its "prefill"
 object, each with its roofline, CPU oracle baseline, end-to-end figure and
 clocks.
 
-Every timed region is one replay of a CUDA graph of the K timed steps,
-bracketed by CUDA events on the launch stream; a spin kernel enqueued just
-before the first event keeps the GPU busy while the host submits the graph,
-so the events see the steps' device time and not the host's launch latency
-(the same number for --steps 20 as for --steps 2000).
+Every timed region is one replay of a CUDA graph holding one untimed step
+and then the K timed steps, with CUDA events recorded inside the graph around
+the timed ones: the start event on a side branch after the untimed step, so
+the first timed step overlaps its predecessor (programmatic dependent launch)
+like every later one, and the events bracket K steps of the steady state,
+free of the graph's start-up and the host's launch latency (the same per-step
+time for --steps 20 as for --steps 2000).  A spin kernel ahead of the replay
+keeps the GPU busy while the host submits the graph.
 
 A step is one pass of the BitLinear forward over one batch of synthetic,
 seeded input: per-token activation quantisation, the ternary x int8
@@ -205,7 +208,7 @@ def workload_identity(workload: str, sweep_m: int = 8, layers: int = 30) -> dict
     raise ValueError(workload)
 
 
-def make_decode(tw, torch, dev, l2_bytes):
+def make_decode(tw, torch, dev, l2_bytes, table_lookup=False):
     import synth
     d = synth.config_inputs("decode")
     W = torch.from_numpy(d["W"]).to(dev)
@@ -219,7 +222,8 @@ def make_decode(tw, torch, dev, l2_bytes):
     Y = torch.empty((1, d["N"]), dtype=torch.bfloat16, device=dev)
 
     def step(i, stream=None):
-        tw.bitnet_w158a8_matmul(X, copies[i % R], gamma, Y=Y, weights_static=True, stream=stream)
+        tw.bitnet_w158a8_matmul(X, copies[i % R], gamma, Y=Y, weights_static=True,
+                                table_lookup=table_lookup, stream=stream)
 
     return dict(
         step=step, kernel_step=step, units_per_step=wbytes, unit="GB/s", scale=1e-9, bound="hbm",
@@ -228,15 +232,16 @@ def make_decode(tw, torch, dev, l2_bytes):
                 "l2": f"inputs larger than L2: {R} rotating weight copies, "
                       f"{R * wbytes / 1e6:.0f} MB >= 3x L2",
                 "timing": "CUDA graph of the timed steps, programmatic dependent launch, "
-                          "weights flagged static"},
-        kernel_key="decode_gemv_M1_K2560_N2560",
+                          "weights flagged static",
+                **({"kernel": "table-lookup comparison kernel"} if table_lookup else {})},
+        kernel_key=None if table_lookup else "decode_gemv_M1_K2560_N2560",
         kernel_files=["ternary_weight_linear_token_b200/csrc/gemv_rows.cu",
                       "ternary_weight_linear_token_b200/csrc/common.cuh"],
         e2e_inputs=lambda: (d["x_bits"].view(np.int16), 2 * d["K"], 2 * d["N"]),
     )
 
 
-def make_sweep(tw, torch, dev, l2_bytes, M=8):
+def make_sweep(tw, torch, dev, l2_bytes, M=8, table_lookup=False):
     """Decode sweep: one step is one decoder layer's four projections (qkv,
     o, up + ReLU^2, down) at M tokens, each a dependent call."""
     import synth
@@ -259,10 +264,12 @@ def make_sweep(tw, torch, dev, l2_bytes, M=8):
         for q in projs:
             tw.bitnet_w158a8_matmul(q["X"], q["copies"][i % R], q["gamma"], relu2=q["relu2"],
                                     Y=q["Y"], workspace=q["ws"], weights_static=True,
-                                    stream=stream)
+                                    table_lookup=table_lookup, stream=stream)
 
     d0 = projs[0]["d"]
-    launches = 4 if M <= 3 else 8  # 4 tokens and more: quantiser + product per projection
+    # 4 tokens and more: quantiser + product per projection (the table-lookup
+    # kernel quantises inside, like the fused one)
+    launches = 4 if (M <= 3 or table_lookup) else 8
     return dict(
         step=step, kernel_step=step, units_per_step=wbytes, unit="GB/s", scale=1e-9, bound="hbm",
         launches_per_step=launches, X=projs[0]["X"], Y=projs[3]["Y"], rotate=R,
@@ -270,7 +277,8 @@ def make_sweep(tw, torch, dev, l2_bytes, M=8):
                 "l2": f"inputs larger than L2: {R} rotating copies of the layer's weights, "
                       f"{R * wbytes / 1e6:.0f} MB >= 3x L2",
                 "timing": "CUDA graph of the timed steps, programmatic dependent launch, "
-                          "weights flagged static"},
+                          "weights flagged static",
+                **({"kernel": "table-lookup comparison kernel"} if table_lookup else {})},
         kernel_key=None, kernel_files=[],
         e2e_inputs=lambda: (d0["x_bits"].view(np.int16), 2 * M * d0["K"], 2 * M * 2560),
     )
@@ -472,33 +480,46 @@ def run_reference(args, world, rank):
     return 0
 
 
-# Spin cycles that keep the GPU busy while the host submits a timed graph:
-# the event pair then brackets the graph's device time alone, whatever the
-# host's launch latency (about 1 ms plus 1 us per graph node at ~2 GHz).
+# Spin cycles that keep the GPU busy while the host submits a timed graph
+# (about 1 ms plus 1 us per graph node at ~2 GHz).
 def spin_cycles(nodes: int) -> int:
     return int(2_000_000 + 2_000 * nodes)
 
 
-def capture(torch, stream, fn, first: int, count: int):
-    """One CUDA graph of `count` calls fn(first + i, stream)."""
+def capture_timed(torch, stream, fn, warm: int, first: int, count: int):
+    """One CUDA graph: an untimed step fn(warm), then `count` timed steps
+    fn(first + i), with a timing event before and after the timed ones.
+
+    The start event is recorded on a side branch of the graph that depends on
+    the untimed step alone, so the first timed step follows that step by
+    programmatic dependent launch exactly as every later step follows its
+    predecessor: the two events bracket `count` steps of the steady state,
+    the same per-step time whether `count` is 20 or 2000, and none of the
+    graph's start-up latency."""
+    ev0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev1 = torch.cuda.Event(enable_timing=True, external=True)
+    side = torch.cuda.Stream(stream.device)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
+        fn(warm, stream)
+        side.wait_stream(stream)
+        ev0.record(side)
         for i in range(count):
             fn(first + i, stream)
-    return g
+        ev1.record(stream)
+        stream.wait_stream(side)
+    return g, ev0, ev1
 
 
-def replay_timed(torch, graph, stream, nodes: int, clocks=None):
-    """Device time (ms) of one replay of `graph`, CUDA events on `stream`.
-    A spin kernel ahead of the first event hides the host's graph submission."""
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+def replay_timed(torch, timed, stream, nodes: int):
+    """Device time (ms) between the events of one replay of a captured timed
+    graph.  A spin kernel ahead of it keeps the GPU busy while the host
+    submits the graph."""
+    g, ev0, ev1 = timed
     with torch.cuda.stream(stream):
         torch.cuda._sleep(spin_cycles(nodes))
-        ev0.record(stream)
-        graph.replay()          # replays on the current stream, i.e. `stream`
-        ev1.record(stream)
-    ev1.synchronize()
+        g.replay()          # replays on the current stream, i.e. `stream`
+    stream.synchronize()
     return ev0.elapsed_time(ev1)
 
 
@@ -509,14 +530,14 @@ def measure(w, tw, torch, args, dev, stream, pg, world, rank, bus):
         for i in range(args.warmup):
             w["step"](i, stream)
     stream.synchronize()
-    graph = capture(torch, stream, w["step"], args.warmup, args.steps)
+    graph = capture_timed(torch, stream, w["step"], args.warmup - 1, args.warmup, args.steps)
     kgraph = None
     if w.get("kernel_step") is not None and w["kernel_step"] is not w["step"]:
-        kgraph = capture(torch, stream, w["kernel_step"], 0, args.steps)
+        kgraph = capture_timed(torch, stream, w["kernel_step"], args.steps, 0, args.steps)
     with torch.cuda.stream(stream):
-        graph.replay()  # one untimed replay of each: first-launch costs of the graphs
+        graph[0].replay()  # one untimed replay of each: first-launch costs of the graphs
         if kgraph is not None:
-            kgraph.replay()
+            kgraph[0].replay()
     stream.synchronize()
 
     if pg:
@@ -551,7 +572,7 @@ def measure(w, tw, torch, args, dev, stream, pg, world, rank, bus):
                 "kernel_us": 1e3 * kms / args.steps,
                 "kernel_timing": ("the tensor-core kernel alone: a CUDA graph of one launch "
                                   "per step on prepared int8 activations and int8 weight "
-                                  "copies, CUDA events on the launch stream")
+                                  "copies, CUDA events around the timed launches")
                 if kgraph is not None else "CUDA-event time of the timed steps"}
 
     # end to end through the public API: pinned host input -> device -> result -> host
@@ -605,6 +626,9 @@ def main():
                     help="chain workload: one persistent kernel per token, or one launch per step")
     ap.add_argument("--no-prefill", action="store_true",
                     help="decode workload: leave out the prefill object of the JSON line")
+    ap.add_argument("--table-lookup", action="store_true",
+                    help="decode and sweep workloads (M <= 8): run the table-lookup comparison "
+                         "kernel instead of the library's default path")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world, rank, local = dist_setup()
@@ -632,6 +656,8 @@ def main():
     extra = {"persistent": args.chain_mode == "persistent"} if args.workload == "chain" else {}
     if args.workload == "sweep":
         extra = {"M": args.sweep_m}
+    if args.table_lookup and args.workload in ("decode", "sweep"):
+        extra["table_lookup"] = True
     stream = torch.cuda.Stream(dev)
     w = MAKERS[args.workload](tw, torch, dev, l2, **extra)
     w["name"] = args.workload
@@ -640,7 +666,7 @@ def main():
     del w
 
     prefill = None
-    if args.workload == "decode" and not args.no_prefill:
+    if args.workload == "decode" and not args.no_prefill and not args.table_lookup:
         # the other half of the metric: the prefill GEMM (M=4096, K=2560,
         # N=6912) with the same timing rules, as its own object
         wp = make_prefill(tw, torch, dev, l2)

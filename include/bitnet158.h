@@ -107,6 +107,19 @@ typedef enum bitnet_epilogue {
  * takes).  A wrong promise gives wrong results, not an error. */
 #define BITNET_FLAG_WEIGHTS_EXPANDED 2u
 
+/* Flag for bitnet_w158a8_matmul: run the table-lookup kernel instead, the
+ * GPU form of the CPU kernels that "Microsoft BitNet 深度研究报告" describes
+ * (技术原理 item 3, 查找表优化; the TL1/TL2 rows of its bitnet.cpp kernel
+ * table): per token, every sum that two ternary weights (one 4-bit nibble of
+ * the packed layout) can select from two activations is tabulated, and each
+ * packed byte then costs two table reads.  Same results, bit for bit, as the
+ * other kernels; kept as a measured comparison (it is slower here: every CTA
+ * builds the whole table for its few rows).  1 <= M <= 8 tokens, any input
+ * dtype, no workspace; shapes whose tables of one token do not fit in shared
+ * memory (K above about 10000) return BITNET_ERR_UNSUPPORTED_SHAPE.  Not
+ * accepted by bitnet_rms_norm_w158a8_matmul. */
+#define BITNET_FLAG_TABLE_LOOKUP 4u
+
 /* ----------------------------------------------------------------------
  * Weight quantisation: absmean ternary codes, packed four per byte.
  * ("Microsoft BitNet 深度研究报告", 技术原理 item 2; 2B4T report write-up,
@@ -157,7 +170,8 @@ bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M
  *   workspace at least bitnet_w158a8_matmul_workspace_size(M, N, K, x_dtype)
  *            bytes (may be NULL when that is 0).  Contents on entry don't
  *            matter; the call may overwrite all of it.
- *   flags    0, or BITNET_FLAG_WEIGHTS_STATIC and/or BITNET_FLAG_WEIGHTS_EXPANDED.
+ *   flags    0, or any of BITNET_FLAG_WEIGHTS_STATIC, BITNET_FLAG_WEIGHTS_EXPANDED,
+ *            BITNET_FLAG_TABLE_LOOKUP.
  * Up to 3 tokens (8 when K % 64 != 0) run one fused kernel and need no
  * workspace.  Otherwise fp32/bf16 input is first quantised into the
  * workspace by the activation quantiser (M*K bytes + 4*M, each rounded up to
@@ -296,12 +310,13 @@ bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, in
  *              overlap any output.
  *   y_norm     bf16 [steps[n-1].N] or NULL: the RMS normalisation of the
  *              last step's output (N % 16 == 0 and N <= 8192 when given).
- *   workspace  >= bitnet_decode_chain_workspace_size(steps, n_steps) bytes,
- *              16-byte aligned.  ZERO-FILLED before the first call; then
- *              passed unchanged to every later call of a chain (the library
- *              keeps a launch counter in it and tags its exchange words with
- *              it).  After a call that reported BITNET_ERR_TIMEOUT, zero it
- *              again.  Two chains must not run concurrently on one workspace.
+ *   workspace  >= bitnet_decode_chain_workspace_size(steps, n_steps) bytes
+ *              (256 + 1152 * n_steps, rounded up to 256), 16-byte aligned.
+ *              ZERO-FILLED before the first call; then passed unchanged to
+ *              every later call of a chain (the library keeps a launch
+ *              counter and per-step arrival counters in it, which only grow).
+ *              After a call that reported BITNET_ERR_TIMEOUT, zero it again.
+ *              Two chains must not run concurrently on one workspace.
  * Per step: packed [N][K/4] and gamma as from bitnet_quantize_weights
  * (packed 16-byte aligned); Y bf16 [N], 16-byte aligned; 1 <= N <= 2^22;
  * K % 64 == 0, 64 <= K <= 8192 and K <= the previous step's N.  Shapes whose

@@ -142,8 +142,10 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
     return BITNET_ERR_INVALID_ARG;
   if (epi != BITNET_EPI_NONE && epi != BITNET_EPI_RELU2) return BITNET_ERR_INVALID_ARG;
   if (y_dtype == BITNET_I32 && epi != BITNET_EPI_NONE) return BITNET_ERR_INVALID_ARG;
-  if ((flags & ~(BITNET_FLAG_WEIGHTS_STATIC | BITNET_FLAG_WEIGHTS_EXPANDED)) != 0)
+  if ((flags & ~(BITNET_FLAG_WEIGHTS_STATIC | BITNET_FLAG_WEIGHTS_EXPANDED |
+                 BITNET_FLAG_TABLE_LOOKUP)) != 0)
     return BITNET_ERR_INVALID_ARG;
+  if ((flags & BITNET_FLAG_TABLE_LOOKUP) != 0 && norm_in) return BITNET_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
   if (bitnet_status st = check_k(K)) return st;
   if (M == 0 || N == 0) return BITNET_OK;
@@ -157,6 +159,8 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
               static_cast<size_t>(M) * N * elem_size(y_dtype)))
     return BITNET_ERR_INVALID_ARG;
   // the normalising variant runs the fused kernel, with no scratch, whenever it can
+  if ((flags & BITNET_FLAG_TABLE_LOOKUP) != 0)  // the comparison kernel: no scratch
+    return lut_supported(M, N, K) ? BITNET_OK : BITNET_ERR_UNSUPPORTED_SHAPE;
   if (!check_workspace) return BITNET_OK;
   const size_t need = norm_in && rows_supported(M, N, K) ? 0 : matmul_workspace(M, N, K, x_dtype);
   if (need > 0) {
@@ -237,9 +241,8 @@ bitnet_status check_chain(const bitnet_chain_step *steps, int n_steps) {
 }
 
 size_t chain_workspace(const bitnet_chain_step *steps, int n_steps) {
-  size_t words = 0;
-  for (int s = 0; s < n_steps; ++s) words += static_cast<size_t>(chain_xch_words(steps[s].N));
-  return align256(kChainWorkspaceHeader + chain_stats_bytes(n_steps) + kChainReplicas * 8 * words);
+  (void)steps;
+  return align256(kChainWorkspaceHeader + chain_sync_bytes(n_steps));
 }
 
 }  // namespace
@@ -344,6 +347,9 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
   if (M == 0 || N == 0) return BITNET_OK;  // empty: pointers may be NULL
   LaunchCtx ctx;
   if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  if ((flags & BITNET_FLAG_TABLE_LOOKUP) != 0)
+    return from_cuda(launch_lut(X, x_dtype, s, packed, gamma, M, N, K, epi == BITNET_EPI_RELU2, Y,
+                                y_dtype, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0, ctx));
   return run_matmul(X, x_dtype, s, packed, gamma, M, N, K, epi == BITNET_EPI_RELU2, Y, y_dtype,
                     workspace, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0,
                     (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0, ctx);

@@ -417,4 +417,89 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w) {
                     unpack_natural(w, 3));
 }
 
+
+// ------------------------------------------------------------ decode dot products
+// The unpack order of one 16-element group of int8 activations in shared
+// memory (16 bytes): the elements that the byte-permute unpack below pairs
+// with selector shifts 0, 16, 2, 18 -- {0,8,1,9}, {2,10,3,11}, {4,12,5,13},
+// {6,14,7,15} -- so elements 0..7 of the group fill bytes 0..7 with the help
+// of 4 bytes from elements 8..11, and vice versa.
+constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
+
+// clamp(round_half_away(x * s), -127, 127) of 8 values, packed as 8 int8
+// in their order (two words, first value in the lowest byte), on the FMA and
+// ALU pipes: the nearest integer (ties to even, the IEEE rounding of the add)
+// is the low byte of x * s + 1.5 * 2^23; a remainder of exactly one half (a
+// tie, found as the chunk's largest |v - r|, which is at most 1/2) is moved
+// away from zero in a rarely taken branch.  The same arithmetic as quant16:
+// within the contract (finite x, s = 127 / max |x|) |x * s| rounds to at
+// most 127, so the clamp never binds and is left out.
+__device__ __forceinline__ uint2 quant8_packed(const float (&x)[8], float s) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
+  uint32_t t[8];
+  float d[8];
+  float dmax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float v = __fmul_rn(x[e], s);
+    const float tf = __fadd_rn(v, kMagic);
+    t[e] = __float_as_uint(tf);
+    d[e] = __fsub_rn(v, __fsub_rn(tf, kMagic));
+    dmax = fmaxf(dmax, fabsf(d[e]));
+  }
+  if (dmax == 0.5f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int q = static_cast<int>(t[e] - 0x4B400000u);
+      if (fabsf(d[e]) == 0.5f && (q == 0 || (d[e] > 0.0f) == (q > 0))) t[e] += d[e] > 0.0f ? 1u : ~0u;
+    }
+  }
+  return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040u), __byte_perm(t[2], t[3], 0x0040u), 0x5410u),
+                    __byte_perm(__byte_perm(t[4], t[5], 0x0040u), __byte_perm(t[6], t[7], 0x0040u), 0x5410u));
+}
+
+// Quantise one 8-element half-group and store it, with the partner lane's
+// help, in the unpack order.  Both lanes of a pair must call this together
+// (the shuffle needs the whole warp); `active` is false past the end of K.
+__device__ __forceinline__ void store_half_group(uint8_t *xrow, int chunk, const float (&v)[8],
+                                                 float sm, bool active) {
+  const uint2 ab = active ? quant8_packed(v, sm) : make_uint2(0u, 0u);
+  const bool lo = (chunk & 1) == 0;  // elements 0..7 of the group (else 8..15)
+  const uint32_t a = ab.x, b = ab.y;
+  // low half sends elements 4..7, high half sends elements 8..11
+  const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? b : a, 1);
+  if (!active) return;
+  uint2 o;
+  if (lo) {  // bytes 0..7: {0,8,1,9}, {2,10,3,11}
+    o.x = __byte_perm(a, other, 0x5140);
+    o.y = __byte_perm(a, other, 0x7362);
+  } else {   // bytes 8..15: {4,12,5,13}, {6,14,7,15}
+    o.x = __byte_perm(other, b, 0x5140);
+    o.y = __byte_perm(other, b, 0x7362);
+  }
+  *reinterpret_cast<uint2 *>(xrow + 8 * chunk) = o;
+}
+
+// The 16 int8 weights of a packed word, as four dp4a operands in the
+// shared-memory K order (selector shifts 0, 16, 2, 18).
+struct Unpacked {
+  int a, b, c, d;
+};
+// The byte permute reads only the low 16 bits of its selector, so one mask
+// of the whole word serves two selectors (shift 0 and 16; shift 2 and 18).
+__device__ __forceinline__ Unpacked unpack_word(uint32_t w) {
+  const uint32_t m0 = w & 0x33333333u, m1 = (w >> 2) & 0x33333333u;
+  return {static_cast<int>(__byte_perm(kTernaryLut, 0u, m0)),
+          static_cast<int>(__byte_perm(kTernaryLut, 0u, m0 >> 16)),
+          static_cast<int>(__byte_perm(kTernaryLut, 0u, m1)),
+          static_cast<int>(__byte_perm(kTernaryLut, 0u, m1 >> 16))};
+}
+__device__ __forceinline__ int dot_word(const Unpacked &q, uint4 x, int acc) {
+  acc = __dp4a(q.a, static_cast<int>(x.x), acc);
+  acc = __dp4a(q.b, static_cast<int>(x.y), acc);
+  acc = __dp4a(q.c, static_cast<int>(x.z), acc);
+  acc = __dp4a(q.d, static_cast<int>(x.w), acc);
+  return acc;
+}
+
 }  // namespace bitnet

@@ -37,7 +37,6 @@ constexpr int kRows = 16;
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kSmemLimit = 227 * 1024;
-constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
 
 struct DecodeParams {
   const void *X;

@@ -30,7 +30,6 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxBlocks = 8;   // 8-row weight blocks per CTA
 constexpr int kHeader = 256;    // mbarrier, gamma / s for 32 tokens
 constexpr int kSmemLimit = 227 * 1024;
-constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
 
 struct MmvParams {
   const int8_t *xq;     // [M][K], unpack order

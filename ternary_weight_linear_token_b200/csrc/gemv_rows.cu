@@ -42,7 +42,6 @@ namespace {
 constexpr int kMaxWarps = 32;
 constexpr int kMaxTok = 8;
 constexpr int kSmemLimit = 227 * 1024;
-constexpr uint32_t kTernaryLut = 0xFFFF0100u;  // code 0 -> 0, 1 -> +1, 2 -> -1, 3 -> -1
 
 struct RowsParams {
   const void *X;
@@ -160,50 +159,6 @@ __device__ __forceinline__ void load8(const void *X, size_t idx, float (&v)[8]) 
       v[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
     }
   }
-}
-
-// Quantise one 8-element half-group and store it, with the partner lane's
-// help, in the unpack order.  Both lanes of a pair must call this together
-// (the shuffle needs the whole warp); `active` is false past the end of K.
-__device__ __forceinline__ void store_half_group(uint8_t *xrow, int chunk, const float (&v)[8],
-                                                 float sm, bool active) {
-  int q[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) q[e] = active ? quant_i8(v[e], sm) : 0;
-  const bool lo = (chunk & 1) == 0;  // elements 0..7 of the group (else 8..15)
-  const uint32_t a = pack4(q[0], q[1], q[2], q[3]);
-  const uint32_t b = pack4(q[4], q[5], q[6], q[7]);
-  // low half sends elements 4..7, high half sends elements 8..11
-  const uint32_t other = __shfl_xor_sync(0xffffffffu, lo ? b : a, 1);
-  if (!active) return;
-  uint2 o;
-  if (lo) {  // bytes 0..7: {0,8,1,9}, {2,10,3,11}
-    o.x = __byte_perm(a, other, 0x5140);
-    o.y = __byte_perm(a, other, 0x7362);
-  } else {   // bytes 8..15: {4,12,5,13}, {6,14,7,15}
-    o.x = __byte_perm(other, b, 0x5140);
-    o.y = __byte_perm(other, b, 0x7362);
-  }
-  *reinterpret_cast<uint2 *>(xrow + 8 * chunk) = o;
-}
-
-// The 16 int8 weights of a packed word, as four dp4a operands in the
-// shared-memory K order (selector shifts 0, 16, 2, 18).
-struct Unpacked {
-  int a, b, c, d;
-};
-__device__ __forceinline__ Unpacked unpack_word(uint32_t w) {
-  return {static_cast<int>(__byte_perm(kTernaryLut, 0u, w & 0x3333u)),
-          static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 16) & 0x3333u)),
-          static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 2) & 0x3333u)),
-          static_cast<int>(__byte_perm(kTernaryLut, 0u, (w >> 18) & 0x3333u))};
-}
-__device__ __forceinline__ int dot_word(const Unpacked &q, uint4 x, int acc) {
-  acc = __dp4a(q.a, static_cast<int>(x.x), acc);
-  acc = __dp4a(q.b, static_cast<int>(x.y), acc);
-  acc = __dp4a(q.c, static_cast<int>(x.z), acc);
-  acc = __dp4a(q.d, static_cast<int>(x.w), acc);
-  return acc;
 }
 
 // x rounded to the input's precision (the normalised input is stored in it).

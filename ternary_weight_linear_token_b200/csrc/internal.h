@@ -50,6 +50,12 @@ cudaError_t launch_rows(const void *X, int x_kind, const float *s, const uint8_t
                         int y_kind, bool weights_static, bool norm, void *Xn,
                         const LaunchCtx &ctx);
 
+// gemv_lut.cu: table-lookup comparison kernel for 1 <= M <= 8 tokens, K % 16 == 0.
+bool lut_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_lut(const void *X, int x_kind, const float *s, const uint8_t *packed,
+                       const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2, void *Y,
+                       int y_kind, bool weights_static, const LaunchCtx &ctx);
+
 // gemv_decode.cu: fused decode kernel, M <= 32, K % 64 == 0.
 bool decode_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_decode(const void *X, int x_kind, const float *s, const uint8_t *packed,
@@ -84,15 +90,13 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
 constexpr int kChainMaxSteps = 256;
 constexpr int kStepRelu2 = 1;
 constexpr int kStepNormIn = 2;
-constexpr size_t kChainWorkspaceHeader = 256;  // launch counter, finished-CTA counter
+constexpr size_t kChainWorkspaceHeader = 256;  // the launch counter at byte 0
 constexpr int kChainMaxCtas = 256;              // CTAs of one chain launch, at most
-// Copies of everything the CTAs exchange (CTA c reads copy c % kChainReplicas),
-// so that fewer SMs poll and load the same L2 lines.
-constexpr int kChainReplicas = 4;
-// Per-step, per-CTA records (two tagged 64-bit words: max |y|, sum y^2), one
-// set per copy, after the header; they double as the CTA's "outputs are out" flag.
-inline size_t chain_stats_bytes(int n_steps) {
-  return static_cast<size_t>(kChainReplicas) * n_steps * kChainMaxCtas * 16;
+// After the header, one 128-byte line per step holding its arrival counter,
+// then per step kChainMaxCtas floats: each CTA's max |y| of the step.
+constexpr size_t kChainLine = 128;
+inline size_t chain_sync_bytes(int n_steps) {
+  return (kChainLine + 4 * static_cast<size_t>(kChainMaxCtas)) * static_cast<size_t>(n_steps);
 }
 struct ChainStep {
   const uint8_t *packed;
@@ -103,11 +107,9 @@ struct ChainStep {
   void *Xn;
 };
 struct ChainPlan {
-  int ctas, slots, slot_bytes, xq_bytes, ystage_bytes;
+  int ctas, slots, slot_bytes, xq_bytes, part_bytes, part_stride;
   size_t smem;
 };
-// 64-bit exchange words of one step's output: two bf16 values each.
-inline int64_t chain_xch_words(int64_t N) { return (N + 1) / 2; }
 int chain_max_k();
 bool chain_plan(const ChainStep *steps, int n_steps, int num_sms, ChainPlan *plan);
 cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &plan,

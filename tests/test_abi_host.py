@@ -70,7 +70,7 @@ def test_matmul_rejects_bad_arguments(tw):
     assert mm(tw, yd=2) == tw.ERR_INVALID_ARG            # int8 output
     assert mm(tw, epi=2) == tw.ERR_INVALID_ARG
     assert mm(tw, yd=3, epi=1) == tw.ERR_INVALID_ARG     # raw int32 with ReLU^2
-    assert mm(tw, flags=4) == tw.ERR_INVALID_ARG         # unknown flag bit
+    assert mm(tw, flags=8) == tw.ERR_INVALID_ARG         # unknown flag bit
     assert mm(tw, M=-1) == tw.ERR_INVALID_ARG
     assert mm(tw, K=0) == tw.ERR_INVALID_ARG
     assert mm(tw, K=40) == tw.ERR_UNSUPPORTED_SHAPE      # not a multiple of 16
@@ -174,14 +174,12 @@ def test_decode_chain_rejects_bad_arguments(tw):
 def test_decode_chain_workspace_size(tw):
     f = tw.lib.bitnet_decode_chain_workspace_size
     layer = [(3840, 2560), (2560, 2560), (6912, 2560), (2560, 6912)]
-    # 256-byte header; then 4 copies of: one 16-byte record per CTA (up to
-    # 256) per step; then 4 copies of: one 8-byte word per two outputs of
-    # every step
-    words = sum((n + 1) // 2 for n, _ in layer)
-    assert f(chain(tw, layer), 4) == (256 + 4 * 4 * 4096 + 4 * 8 * words + 255) // 256 * 256
-    assert f(chain(tw, [(333, 64)]), 1) == 22016     # 256 + 16384 + 5344 = 21984, rounded up
+    # 256-byte header (the launch counter); then one 128-byte line per step
+    # for its arrival counter, then per step 256 floats (each CTA's max |y|)
+    assert f(chain(tw, layer), 4) == (256 + 4 * 1152 + 255) // 256 * 256
+    assert f(chain(tw, [(333, 64)]), 1) == 1536      # 256 + 1152 = 1408, rounded up
     assert f(chain(tw, [(64, 40)]), 1) == 0          # invalid descriptors
-    assert f(chain(tw, layer * 30), 120) > 0
+    assert f(chain(tw, layer * 30), 120) == 256 + 120 * 1152
 
 
 def test_rms_norm_matmul_rejects_bad_arguments(tw):
@@ -199,6 +197,17 @@ def test_rms_norm_matmul_rejects_bad_arguments(tw):
     assert call(Xn=C.c_void_p(0x10000000)) == tw.ERR_INVALID_ARG  # X_normed overlapping X
     assert call(Xn=C.c_void_p(0x30000000)) == tw.ERR_INVALID_ARG  # X_normed overlapping Y
     assert call(M=0) == tw.OK
+
+
+def test_table_lookup_flag_checks(tw):
+    """The table-lookup comparison kernel takes 1..8 tokens and no workspace;
+    larger M is an unsupported shape, and the normalising variant refuses
+    the flag.  All decided before any device access."""
+    assert mm(tw, M=9, K=64, flags=4) == tw.ERR_UNSUPPORTED_SHAPE
+    assert mm(tw, M=1, N=8, K=1 << 20, flags=4) == tw.ERR_UNSUPPORTED_SHAPE  # tables too big
+    assert mm(tw, M=0, flags=4) == tw.OK
+    f = tw.lib.bitnet_rms_norm_w158a8_matmul
+    assert f(A, 1, None, B, G, 4, 8, 64, 0, Cc, 1, None, 0, 4, None) == tw.ERR_INVALID_ARG
 
 
 def test_matmul_path_query(tw):

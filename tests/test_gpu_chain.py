@@ -2,10 +2,12 @@
 link by link: every step's bf16 output must equal the oracle's BitLinear of
 the step's actual bf16 input (bit-exact); a normalised input (BITNET_STEP_NORM_IN)
 must be within 1 bf16 ulp of the oracle's RMS normalisation of the previous
-output, and the oracle's BitLinear is then fed the kernel's own normalised
-values.  Shapes cover odd N (a half-filled last exchange word), K smaller than
-the previous N, CTAs that own no row of a step (N < number of SMs), both
-epilogues, repeated launches on one workspace and CUDA-graph replay."""
+output (both sum the squares in fp64 and round the factor once, so in
+practice it is bit-identical), and the oracle's BitLinear is then fed the
+kernel's own normalised values.  Shapes cover odd N (a half-filled last
+32-bit store), K smaller than the previous N, CTAs that own no row of a step
+(N < number of SMs), both epilogues, repeated launches on one workspace and
+CUDA-graph replay; and the configured 30-layer stack in both chain forms."""
 
 from __future__ import annotations
 
@@ -158,18 +160,19 @@ def test_decode_chain_matches_per_launch_chain(tw):
 
 def test_decode_chain_bounded_wait_reports_timeout(tw):
     """A wait that never completes gives up (about 2 s) and is reported, with
-    no fault: the finished-CTA counter in a zero-filled workspace starts at
-    2^30, above the count CTA 0 waits for at the end (the number of CTAs), and
-    only grows, so that count never appears.  (A start of 1 would not do: the
-    count then passes through the awaited value just before the last CTA
-    counts itself out, and CTA 0 may see it.)  The links computed before that
-    are still right, the device status is BITNET_ERR_TIMEOUT, and the launch
-    counter is not advanced (zero the workspace again after a timeout, as the
-    header says)."""
+    no fault: the last step's arrival counter in a zero-filled workspace
+    starts at 2^30, so it never equals the count CTA 0 waits for at the end
+    (the number of CTAs), and only grows, so that count never appears.  (A
+    start below the awaited count would not do: the count could pass through
+    it.)  Only CTA 0 waits on the last step's counter; every link is
+    computed before that and is still right, the device status is
+    BITNET_ERR_TIMEOUT, and the launch counter is not advanced (zero the
+    workspace again after a timeout, as the header says)."""
     steps, Ws = build_chain(tw, SHAPES_A[:2], 31)
     arr = tw.bitnet_decode_chain_steps(steps)
     ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
-    ws.view(torch.int32)[32] = 1 << 30  # byte 128: the finished-CTA counter
+    last = len(steps) - 1
+    ws.view(torch.int32)[(256 + 128 * last) // 4] = 1 << 30  # the last step's arrival counter
     assert tw.bitnet_get_device_status() == tw.OK
     x0 = x0_bits(SHAPES_A[0][1], 7)
     tw.bitnet_decode_chain(arr, bf16_t(x0), ws)
@@ -273,15 +276,22 @@ def test_stack30_per_launch_links_and_end_to_end(tw, stack30):
 
 def test_stack30_persistent_links(tw, stack30):
     """The persistent form (one bitnet_decode_chain launch per token, 120
-    steps, the 8-slot weight ring wrapping 15 times) of the 30-layer stack:
-    every link against the oracle, on two launches in a row (the second
-    with another input) and on a CUDA-graph replay."""
+    steps, the weight ring of shared-memory slots wrapping many times) of
+    the 30-layer stack: every link against the oracle and the whole first
+    run against the oracle's own run (as for the per-launch form), on two
+    launches in a row (the second with another input) and on a CUDA-graph
+    replay."""
     chain, x0 = stack30["pers"], stack30["x0"]
     for r in range(2):
         bits = x0["x_bits"] if r == 0 else x0_bits(2560, 77)
         chain.run(bf16_t(bits).view(1, -1))
         torch.cuda.synchronize()
-        check_stack(chain, stack30["oracle"], bits)
+        exact = check_stack(chain, stack30["oracle"], bits)
+        assert exact >= 29, exact
+        if r == 0 and exact == 30:  # the whole run equals the oracle's own run
+            for li, (bufs, want) in enumerate(zip(chain.outs, stack30["want"])):
+                for pi in range(5):
+                    assert np.array_equal(bf16_bits_of(bufs[pi]), want[pi]), (li, pi)
     eager = [bf16_bits_of(b).copy() for bufs in chain.outs for b in bufs]
     chain.capture()
     for bufs in chain.outs:

@@ -128,11 +128,13 @@ SHAPES = [
 ]
 
 
-def _run_all_outputs(tw, Xd, sd, packed_d, gamma_d, M, N, K, want_acc, s_o, gamma_o):
+def _run_all_outputs(tw, Xd, sd, packed_d, gamma_d, M, N, K, want_acc, s_o, gamma_o,
+                     table_lookup=False):
     exact = {}
     for out_dtype, relu2 in ((torch.int32, False), (torch.float32, False), (torch.float32, True),
                              (torch.bfloat16, False), (torch.bfloat16, True)):
-        Y = tw.bitnet_w158a8_matmul(Xd, packed_d, gamma_d, s=sd, relu2=relu2, out_dtype=out_dtype)
+        Y = tw.bitnet_w158a8_matmul(Xd, packed_d, gamma_d, s=sd, relu2=relu2, out_dtype=out_dtype,
+                                    table_lookup=table_lookup)
         torch.cuda.synchronize()
         if out_dtype == torch.int32:
             assert np.array_equal(np_of(Y), want_acc), "int32 accumulators differ"
@@ -169,6 +171,36 @@ def test_matmul_parity(tw, M, N, K, xdtype):
     acc_o = ref.matmul_acc(xq_o, packed_o, N, K)
     exact = _run_all_outputs(tw, Xd, sd, packed_d, gamma_d, M, N, K, acc_o, s_o, gamma_o)
     assert all(exact.values()), f"within tolerance but not bit-identical: {exact}"
+
+
+# the table-lookup comparison kernel: 1..8 tokens, several CTAs' rows, K
+# ragged against the 32-lane word loop, K of the down projection (one
+# token's tables per batch), more tokens than fit in one table batch
+LUT_SHAPES = [(1, 2560, 2560), (2, 275, 320), (3, 17, 64), (4, 40, 48), (8, 160, 2560),
+              (5, 100, 6912), (1, 19, 2576), (8, 6912, 2560), (7, 3000, 80)]
+
+
+@pytest.mark.parametrize("M,N,K", LUT_SHAPES)
+@pytest.mark.parametrize("xdtype", ["f32", "bf16", "i8"])
+def test_table_lookup_kernel_parity(tw, M, N, K, xdtype):
+    """The table-lookup kernel (BITNET_FLAG_TABLE_LOOKUP) against the oracle:
+    int32 accumulators and every output dtype bit-exact."""
+    rng = np.random.default_rng(M * 104729 + N * 17 + K)
+    W = synth.latent_weights(rng, N, K)
+    x = rng.standard_t(3, (M, K)).astype(np.float32)
+    packed_d, gamma_d, packed_o, gamma_o = quantize_weights_both(W)
+    if xdtype == "i8":
+        xq_o, s_o = ref.quantize_act(x)
+        Xd, sd = torch.from_numpy(xq_o).to(DEV), torch.from_numpy(s_o).to(DEV)
+    else:
+        Xd, xexact = as_x(x, xdtype)
+        sd = None
+        xq_o, s_o = ref.quantize_act(xexact)
+    acc_o = ref.matmul_acc(xq_o, packed_o, N, K)
+    exact = _run_all_outputs(tw, Xd, sd, packed_d, gamma_d, M, N, K, acc_o, s_o, gamma_o,
+                             table_lookup=True)
+    assert all(exact.values()), f"within tolerance but not bit-identical: {exact}"
+    assert tw.bitnet_get_device_status() == tw.OK
 
 
 def test_matmul_degenerate(tw):
@@ -374,6 +406,41 @@ def test_quantize_act_rounding_near_every_tie(tw):
     wq, ws = ref.quantize_act(x)
     assert np.all(ws == np.float32(1.0)) and np.array_equal(np_of(sc), ws)
     assert np.array_equal(np_of(xq), wq)
+
+
+def test_fused_prologue_rounding_near_every_tie(tw):
+    """The quantiser inside the fused few-token kernel, seen directly: W is
+    the K x K identity (gamma = 1/K, every diagonal code +1, the rest 0), so
+    the int32 accumulators are the int8 activations themselves.  Rows hold
+    every tie k + 0.5 (k = -127..126) with the 64 floats on each side and
+    max |x| = 127 (s = 1 exactly), 1..3 tokens per call (the fused path), fp32
+    and bf16 input; every accumulator must equal the oracle's quantised
+    activation."""
+    K = 4096
+    vals = []
+    for k in range(-127, 127):
+        t = np.float32(k + 0.5)
+        lo = hi = t
+        vals.append(t)
+        for _ in range(64):
+            lo = np.nextafter(lo, np.float32(-np.inf), dtype=np.float32)
+            hi = np.nextafter(hi, np.float32(np.inf), dtype=np.float32)
+            vals += [lo, hi]
+    vals = np.array(vals, dtype=np.float32)
+    vals = vals[np.abs(vals) <= 127.0]
+    rows = (vals.size + K - 2) // (K - 1)
+    body = np.resize(vals, rows * (K - 1)).reshape(rows, K - 1)
+    x = np.concatenate([np.full((rows, 1), 127.0, np.float32), body], axis=1)
+    pd, gd = tw.bitnet_quantize_weights(f32_t(np.eye(K, dtype=np.float32)))
+    for dt in ("f32", "bf16"):
+        for r0 in range(0, rows, 3):
+            xs = x[r0:r0 + 3]
+            Xd, xexact = as_x(xs, dt)
+            assert tw.bitnet_w158a8_matmul_path(xs.shape[0], K, K, Xd.dtype) == tw.PATH_ROWS
+            acc = tw.bitnet_w158a8_matmul(Xd, pd, gd, out_dtype=torch.int32)
+            torch.cuda.synchronize()
+            want, _ = ref.quantize_act(xexact)
+            assert np.array_equal(np_of(acc), want.astype(np.int32)), (dt, r0)
 
 
 # (M, N, K, input dtype, ReLU^2): one-launch fused path for M <= 8, a
