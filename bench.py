@@ -284,7 +284,7 @@ def make_sweep(tw, torch, dev, l2_bytes, M=8, table_lookup=False):
     )
 
 
-def make_prefill(tw, torch, dev, l2_bytes):
+def make_prefill(tw, torch, dev, l2_bytes, prep_in_kernel=False):
     import synth
     d = synth.config_inputs("prefill")
     M, N, K = d["M"], d["N"], d["K"]
@@ -305,7 +305,8 @@ def make_prefill(tw, torch, dev, l2_bytes):
     def step(i, stream=None):
         j = i % R
         tw.bitnet_w158a8_matmul(Xs[j], Ps[j], gamma, Y=Ys[j], workspace=wss[j],
-                                weights_static=True, stream=stream)
+                                weights_static=True, prep_in_kernel=prep_in_kernel,
+                                stream=stream)
 
     # The tensor-core kernel alone: int8 activations (natural K order) with
     # their scales, and per set a workspace whose int8 weight copy a first,
@@ -333,8 +334,10 @@ def make_prefill(tw, torch, dev, l2_bytes):
         Y=Ys[0], path=tw.bitnet_w158a8_matmul_path(M, N, K, torch.bfloat16),
         config={**workload_identity("prefill"),
                 "l2": f"inputs larger than L2: {R} rotating input/output sets",
-                "timing": "CUDA graph; step = activation quantiser (the weights' expansion to "
-                          "int8 scratch runs in the same launch) + tcgen05 kernel"},
+                "timing": ("CUDA graph; step = counter reset + tcgen05 kernel that quantises the "
+                           "activations and expands the weights itself" if prep_in_kernel else
+                           "CUDA graph; step = activation quantiser (the weights' expansion to "
+                           "int8 scratch runs in the same launch) + tcgen05 kernel")},
         kernel_key="prefill_tcgen05_M4096_K2560_N6912",
         kernel_files=["ternary_weight_linear_token_b200/csrc/gemm_prefill.cu",
                       "ternary_weight_linear_token_b200/csrc/common.cuh"],
@@ -626,6 +629,9 @@ def main():
                     help="chain workload: one persistent kernel per token, or one launch per step")
     ap.add_argument("--no-prefill", action="store_true",
                     help="decode workload: leave out the prefill object of the JSON line")
+    ap.add_argument("--prep-in-kernel", action="store_true",
+                    help="prefill workload: the tensor-core kernel prepares its own operands "
+                         "(comparison form)")
     ap.add_argument("--table-lookup", action="store_true",
                     help="decode and sweep workloads (M <= 8): run the table-lookup comparison "
                          "kernel instead of the library's default path")
@@ -658,6 +664,8 @@ def main():
         extra = {"M": args.sweep_m}
     if args.table_lookup and args.workload in ("decode", "sweep"):
         extra["table_lookup"] = True
+    if args.prep_in_kernel and args.workload == "prefill":
+        extra["prep_in_kernel"] = True
     stream = torch.cuda.Stream(dev)
     w = MAKERS[args.workload](tw, torch, dev, l2, **extra)
     w["name"] = args.workload

@@ -120,6 +120,16 @@ typedef enum bitnet_epilogue {
  * accepted by bitnet_rms_norm_w158a8_matmul. */
 #define BITNET_FLAG_TABLE_LOOKUP 4u
 
+/* Flag for bitnet_w158a8_matmul: on the tensor-core path, let the tensor-core
+ * kernel prepare its operands itself while its tiles run (extra warps
+ * quantise the token rows and expand the weight rows, block by block; a
+ * tile's loads wait for its blocks), instead of the separate quantiser
+ * launch that precedes it by default.  Same results, bit for bit.  Kept as a
+ * measured comparison: on B200 it is slower (a handful of preparing warps
+ * per SM cannot stream the operands as fast as a dedicated launch over the
+ * whole GPU, so the tiles wait).  Ignored on the other paths. */
+#define BITNET_FLAG_PREP_IN_KERNEL 8u
+
 /* ----------------------------------------------------------------------
  * Weight quantisation: absmean ternary codes, packed four per byte.
  * ("Microsoft BitNet 深度研究报告", 技术原理 item 2; 2B4T report write-up,
@@ -171,15 +181,16 @@ bitnet_status bitnet_quantize_act(const void *X, bitnet_dtype x_dtype, int64_t M
  *            bytes (may be NULL when that is 0).  Contents on entry don't
  *            matter; the call may overwrite all of it.
  *   flags    0, or any of BITNET_FLAG_WEIGHTS_STATIC, BITNET_FLAG_WEIGHTS_EXPANDED,
- *            BITNET_FLAG_TABLE_LOOKUP.
+ *            BITNET_FLAG_TABLE_LOOKUP, BITNET_FLAG_PREP_IN_KERNEL.
  * Up to 3 tokens (8 when K % 64 != 0) run one fused kernel and need no
  * workspace.  Otherwise fp32/bf16 input is first quantised into the
  * workspace by the activation quantiser (M*K bytes + 4*M, each rounded up to
  * 256); then 4..32 tokens run an int8 mma.sync kernel and larger M the
  * tcgen05 tensor-core kernel, which first expands the packed weights to int8
  * in the workspace (N*K more bytes, rounded up to 256; needed for int8 input
- * too).  The weights in HBM stay packed; the int8 copy is scratch of the
- * call.
+ * too), followed by the readiness counters of BITNET_FLAG_PREP_IN_KERNEL
+ * (32 bytes per 128 tokens and per 256 output features, rounded up to 256).
+ * The weights in HBM stay packed; the int8 copy is scratch of the call.
  * ---------------------------------------------------------------------- */
 size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype);
 
@@ -311,7 +322,7 @@ bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, in
  *   y_norm     bf16 [steps[n-1].N] or NULL: the RMS normalisation of the
  *              last step's output (N % 16 == 0 and N <= 8192 when given).
  *   workspace  >= bitnet_decode_chain_workspace_size(steps, n_steps) bytes
- *              (256 + 1152 * n_steps, rounded up to 256), 16-byte aligned.
+ *              (256 + 256 * n_steps, rounded up to 256), 16-byte aligned.
  *              ZERO-FILLED before the first call; then passed unchanged to
  *              every later call of a chain (the library keeps a launch
  *              counter and per-step arrival counters in it, which only grow).

@@ -34,6 +34,7 @@ EPI_NONE, EPI_RELU2 = 0, 1
 FLAG_WEIGHTS_STATIC = 1
 FLAG_WEIGHTS_EXPANDED = 2
 FLAG_TABLE_LOOKUP = 4
+FLAG_PREP_IN_KERNEL = 8
 PATH_NONE, PATH_ROWS, PATH_MMA_TOKENS, PATH_MMA_WEIGHTS, PATH_TENSOR_CORE, PATH_GENERIC = range(6)
 PATH_NAMES = {PATH_NONE: "none", PATH_ROWS: "rows", PATH_MMA_TOKENS: "mma_tokens",
               PATH_MMA_WEIGHTS: "mma_weights", PATH_TENSOR_CORE: "tensor_core",
@@ -188,13 +189,14 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
                          out_dtype: torch.dtype = torch.bfloat16, Y: torch.Tensor | None = None,
                          workspace: torch.Tensor | None = None, weights_static: bool = False,
                          weights_expanded: bool = False, table_lookup: bool = False,
-                         stream=None) -> torch.Tensor:
+                         prep_in_kernel: bool = False, stream=None) -> torch.Tensor:
     """Y = BitLinear(X).  X is fp32/bf16 [M, K] (quantised inside the call) or
     int8 xq [M, K] with its scales ``s`` [M].  out_dtype fp32/bf16, or int32
     for the raw accumulators (relu2 must then be False).  ``weights_expanded``
     promises that ``workspace`` still holds the int8 weight copy of an
     earlier tensor-core-path call with the same weights and input kind;
-    ``table_lookup`` runs the table-lookup comparison kernel (M <= 8)."""
+    ``table_lookup`` runs the table-lookup comparison kernel (M <= 8);
+    ``prep_in_kernel`` the tensor-core kernel that prepares its own operands."""
     _dev(X, "X", (torch.float32, torch.bfloat16, torch.int8))
     _dev(packed, "packed", (torch.uint8,))
     _dev(gamma, "gamma", (torch.float32,))
@@ -216,7 +218,8 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
                                   _DTYPE[Y.dtype], _ptr(workspace), ws_bytes,
                                   (FLAG_WEIGHTS_STATIC if weights_static else 0)
                                   | (FLAG_WEIGHTS_EXPANDED if weights_expanded else 0)
-                                  | (FLAG_TABLE_LOOKUP if table_lookup else 0),
+                                  | (FLAG_TABLE_LOOKUP if table_lookup else 0)
+                                  | (FLAG_PREP_IN_KERNEL if prep_in_kernel else 0),
                                   _stream(stream))
     _check(st, "bitnet_w158a8_matmul")
     return Y

@@ -125,7 +125,9 @@ size_t matmul_workspace(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   if (use_rows(M, N, K, x_dtype)) return 0;
   const size_t act = x_dtype == BITNET_I8 ? 0 : act_scratch(M, K);
-  return act + (use_prefill(M, N, K, x_dtype) ? align256(prefill_weight_bytes(N, K)) : 0);
+  return act + (use_prefill(M, N, K, x_dtype) ? align256(prefill_weight_bytes(N, K)) +
+                                                    align256(prefill_ready_bytes(M, N))
+                                              : 0);
 }
 
 // Argument checks of bitnet_w158a8_matmul (and of its normalising variant,
@@ -143,7 +145,7 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
   if (epi != BITNET_EPI_NONE && epi != BITNET_EPI_RELU2) return BITNET_ERR_INVALID_ARG;
   if (y_dtype == BITNET_I32 && epi != BITNET_EPI_NONE) return BITNET_ERR_INVALID_ARG;
   if ((flags & ~(BITNET_FLAG_WEIGHTS_STATIC | BITNET_FLAG_WEIGHTS_EXPANDED |
-                 BITNET_FLAG_TABLE_LOOKUP)) != 0)
+                 BITNET_FLAG_TABLE_LOOKUP | BITNET_FLAG_PREP_IN_KERNEL)) != 0)
     return BITNET_ERR_INVALID_ARG;
   if ((flags & BITNET_FLAG_TABLE_LOOKUP) != 0 && norm_in) return BITNET_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
@@ -175,7 +177,7 @@ bitnet_status check_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
 bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
                          const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
                          int64_t K, bool relu2, void *Y, bitnet_dtype y_dtype, void *workspace,
-                         bool wstatic, bool expanded, const LaunchCtx &ctx) {
+                         bool wstatic, bool expanded, bool prep_in_kernel, const LaunchCtx &ctx) {
   if (use_rows(M, N, K, x_dtype))
     return from_cuda(launch_rows(X, x_dtype, s, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                  wstatic, false, nullptr, ctx));
@@ -185,19 +187,40 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
   const bool prefill = use_prefill(M, N, K, x_dtype) && prefill_supported(M, N, K);
   const int8_t *xq = static_cast<const int8_t *>(X);
   const float *sq = s;
-  ExpandJob expand;  // the tensor-core path's int8 weights, after the activation scratch
+  int8_t *wxq = static_cast<int8_t *>(workspace);
+  float *ws = from_float ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                                     align256(static_cast<size_t>(M) * K))
+                         : nullptr;
+  // the tensor-core path's int8 weights follow the activation scratch, then
+  // the readiness counters of its in-kernel form
+  int8_t *w8 = prefill ? static_cast<int8_t *>(workspace) + (from_float ? act_scratch(M, K) : 0)
+                       : nullptr;
+  if (prefill && prep_in_kernel) {
+    // The tensor-core kernel prepares its own operands while it runs: it
+    // quantises fp32/bf16 activations into the workspace (in the K order of
+    // its weight unpack) and expands the packed weights after them (unless
+    // the caller vouches for an earlier expansion).
+    PrefillPrep prep;
+    if (from_float) {
+      prep.X = X;
+      prep.x_kind = x_dtype;
+      xq = wxq;
+      sq = ws;
+    }
+    if (!expanded) prep.packed = packed;
+    prep.ready = reinterpret_cast<unsigned *>(w8 + align256(prefill_weight_bytes(N, K)));
+    return from_cuda(launch_prefill(xq, sq, w8, gamma, M, N, K, relu2, Y, y_dtype, ctx, &prep));
+  }
+  ExpandJob expand;  // the tensor-core path's weight expansion, unless the caller vouches for one
   if (prefill) {
     expand.packed = packed;
-    expand.w8 = static_cast<int8_t *>(workspace) + (from_float ? act_scratch(M, K) : 0);
-    expand.words = expanded ? 0 : N * (K / 16);  // the caller vouches for an earlier expansion
+    expand.w8 = w8;
+    expand.words = expanded ? 0 : N * (K / 16);
   }
   if (from_float) {
     // The prefill and mmv kernels take the quantiser's output in the K order
     // of their fast weight unpack; the generic kernel wants natural order.
     // The weight expansion rides in the quantiser's launch.
-    int8_t *wxq = static_cast<int8_t *>(workspace);
-    float *ws = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                          align256(static_cast<size_t>(M) * K));
     cudaError_t e = launch_quantize_act(X, x_dtype, M, K, wxq, ws, prefill || mmv, ctx, expand);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     xq = wxq;
@@ -206,13 +229,13 @@ bitnet_status run_matmul(const void *X, bitnet_dtype x_dtype, const float *s,
     // the caller's int8 activations are in natural K order
     if (launch_expand_weights(expand, false, ctx) != cudaSuccess) return BITNET_ERR_CUDA;
   }
+  if (prefill)
+    return from_cuda(launch_prefill(xq, sq, w8, gamma, M, N, K, relu2, Y, y_dtype, ctx));
   if (mmv)
     return from_cuda(launch_mmv(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, wstatic, ctx));
   if (decode)
     return from_cuda(launch_decode(xq, BITNET_I8, sq, packed, gamma, M, N, K, relu2, Y, y_dtype,
                                    wstatic, ctx));
-  if (prefill)
-    return from_cuda(launch_prefill(xq, sq, expand.w8, gamma, M, N, K, relu2, Y, y_dtype, ctx));
   return from_cuda(launch_generic(xq, sq, packed, gamma, M, N, K, relu2, Y, y_dtype, ctx));
 }
 
@@ -352,7 +375,8 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                 y_dtype, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0, ctx));
   return run_matmul(X, x_dtype, s, packed, gamma, M, N, K, epi == BITNET_EPI_RELU2, Y, y_dtype,
                     workspace, (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0,
-                    (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0, ctx);
+                    (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0,
+                    (flags & BITNET_FLAG_PREP_IN_KERNEL) != 0, ctx);
 }
 
 bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype, void *X_normed,
@@ -384,7 +408,8 @@ bitnet_status bitnet_rms_norm_w158a8_matmul(const void *X, bitnet_dtype x_dtype,
                                  wstatic, true, X_normed, ctx));
   if (launch_rms_norm(X, x_dtype, M, K, X_normed, x_dtype, ctx) != cudaSuccess) return BITNET_ERR_CUDA;
   return run_matmul(X_normed, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y, y_dtype,
-                    workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0, ctx);
+                    workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0,
+                    (flags & BITNET_FLAG_PREP_IN_KERNEL) != 0, ctx);
 }
 
 bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, int64_t K, void *Y,

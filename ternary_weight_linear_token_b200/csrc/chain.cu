@@ -11,27 +11,29 @@
 //     every projection's packed rows for this CTA into a ring of shared-memory
 //     slots (one bulk copy per projection, L2 evict-first) as far ahead as the
 //     ring allows, while the consumer warps are still on earlier links.
-//   * A link's outputs go straight to that step's output buffer.  Each CTA,
-//     once its outputs of step s are stored, writes the largest |y| among
-//     them (over the part the next step reads) to its slot of the step's
-//     maxima, and then adds one to the step's arrival counter with release
+//   * A link's outputs go straight to that step's output buffer, each warp
+//     storing its finished rows at once.  Each CTA then folds the largest |y|
+//     among them (over the part the next step reads) into one 64-bit word
+//     per step with an atomic max (the launch's tag in the high half, the
+//     float's bits in the low half: non-negative floats order as their bit
+//     patterns, so the maximum is exact and independent of the order of the
+//     CTAs), and adds one to the step's arrival counter with release
 //     semantics.
 //   * Before step s + 1, one thread per CTA polls that counter (one word on
 //     its own line) until every CTA has arrived; then every thread loads its
-//     part of the input vector and every warp the slots of all CTAs, in one
-//     round trip, and each warp reduces the maxima itself (exact in any
-//     order).  Where a layer starts (the weightless RMS normalisation), every
-//     CTA also sums the squares of the loaded input in fp64, all in the same
-//     fixed order, so all CTAs normalise identically.
+//     part of the input vector and the max word, in one round trip.  Where a
+//     layer starts (the weightless RMS normalisation), every CTA also sums
+//     the squares of the loaded input in fp64, all in the same fixed order,
+//     so all CTAs normalise identically.
 //   * Per link, each CTA quantises the whole input to int8 exactly as
 //     bitnet_quantize_act does and computes its balanced range of output
 //     features with the byte-permute unpack and dp4a, in the same int32
 //     arithmetic and with the same epilogue as bitnet_w158a8_matmul.  The
-//     16 consumer warps form a grid: ks slices of K (as many as keep 32 lanes
-//     busy, at most 16) times 16 / ks groups of rows; a lane loads each of its
-//     activation chunks once and uses it for all of its warp's rows, so the
-//     shared-memory traffic per step is about one pass over the weights.
-//     Warp 0 adds the slices' partial sums, applies the epilogue and stores.
+//     16 consumer warps form a grid, chosen per step: ks slices of K times
+//     16 / ks groups of rows, the split that gives the busiest warp the
+//     fewest dot products; a lane loads each of its activation chunks once
+//     per pass of up to 4 rows.  With one slice a warp finishes its rows
+//     itself; otherwise warp 0 adds the slices' partial sums.
 //   * The counters only grow: launch T (T = the launch counter kept in the
 //     workspace, plus one) waits for T * ctas arrivals; CTA 0 advances the
 //     launch counter once all CTAs have passed the last step, so graph
@@ -54,7 +56,7 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr int kHeader = 1024;
 constexpr int kBarConsumers = 1;            // named barrier of the consumer warps
 constexpr int kChunks = 2;                  // 8-element input chunks per thread: K <= 8192
-constexpr int kRowsPerPass = 16;            // rows a warp carries at once in the dot products
+constexpr int kRowsPerPass = 4;             // rows a warp carries at once in the dot products
 
 __host__ __device__ constexpr int align128(int n) { return (n + 127) / 128 * 128; }
 // Shared-memory copies made once at the start: the step descriptors, every
@@ -78,15 +80,15 @@ struct ChainP {
   uint16_t *y_norm;
   unsigned *epoch;
   unsigned *arrive;           // [n_steps], one per 128-byte line
-  float *maxima;              // [n_steps][kMaxCtas]: each CTA's max |y| of the step
+  unsigned long long *amax;   // [n_steps], one per 128-byte line: tag << 32 | max |y| bits
   int *status;
   int n_steps, ctas, slots, slot_bytes, xq_bytes, part_bytes, part_stride, y_norm_n;
   StepP steps[kChainMaxSteps];
 };
 
-__device__ __forceinline__ float ld_cg_f32(const float *p) {
-  float v;
-  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
@@ -184,13 +186,22 @@ __device__ __forceinline__ bool wait_or_stop(uint64_t *bar, uint32_t parity,
   }
 }
 
-// K slices of the consumer warp grid for rows of `words` packed words: as
-// many as keep all 32 lanes of a warp busy (at least 32 words per slice), at
-// most one per warp.
-__host__ __device__ inline int k_slices(int words) {
-  int ks = kCWarps;
-  while (ks > 1 && words < 32 * ks) ks >>= 1;
-  return ks;
+// K slices of the consumer warp grid for `rows` rows of `words` packed
+// words: the power of two ks (1..16; 16 / ks groups of rows) that gives the
+// busiest warp the fewest dot products of a packed word, ceil(rows / rg)
+// rows times ceil(words / (32 ks)) words per lane; the fewest slices among
+// equals.
+__device__ __forceinline__ int k_slices(int rows, int words) {
+  int best = 1, cost = 0x7fffffff;
+  for (int ks = 1; ks <= kCWarps; ks <<= 1) {
+    const int rg = kCWarps / ks;
+    const int c = ((rows + rg - 1) / rg) * ((words + 32 * ks - 1) / (32 * ks));
+    if (c < cost) {
+      cost = c;
+      best = ks;
+    }
+  }
+  return best;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constant__ ChainP P) {
@@ -199,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + 64);          // [kMaxSlots]
   float *red_a = reinterpret_cast<float *>(smem + 128);               // [kCWarps]
   double *red_s = reinterpret_cast<double *>(smem + 192);             // [kCWarps]
+  float *red_max = reinterpret_cast<float *>(smem + 384);             // [kCWarps]
   volatile int *stop = reinterpret_cast<volatile int *>(smem + 320);
   int *issued_sh = reinterpret_cast<int *>(smem + 324);
   int *consumed_sh = reinterpret_cast<int *>(smem + 328);
@@ -299,11 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       }
       float a;
       if (s > 0) {
-        // max |x|: the producers' maxima, one per CTA, reduced by each warp
-        const float *mx = P.maxima + static_cast<size_t>(s - 1) * kMaxCtas;
-        float m = 0.0f;
-        for (int c = lane; c < P.ctas; c += 32) m = fmaxf(m, ld_cg_f32(mx + c));
-        a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+        // the exact max |x| the producers folded together (tag checked)
+        const unsigned long long m = ld_relaxed_u64(P.amax + static_cast<size_t>(s - 1) * 16);
+        a = static_cast<unsigned>(m >> 32) == tag ? __uint_as_float(static_cast<uint32_t>(m)) : 0.0f;
       } else {
         float la = 0.0f;
 #pragma unroll
@@ -371,7 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       const bool have_w = __all_sync(0xffffffffu, mbar_wait(full + slot, phase, P.status));
       const int r0 = rr[s].x, rows = rr[s].y - r0;
       const int words = d.K >> 4;  // packed 32-bit words per row
-      const int ks = k_slices(words), rg = kCWarps / ks;
+      const int ks = k_slices(rows, words), rg = kCWarps / ks;
+      const bool last = s + 1 == P.n_steps;
+      const int k_next = last ? 0 : tab[s + 1].K;
+      const bool relu2 = (d.flags & kStepRelu2) != 0;
+      float wmax = 0.0f;  // this warp's max |y| over stored rows that the next step reads
       if (have_w) {
         consumed = s + 1;
         const uint32_t *wsl =
@@ -396,7 +410,15 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
             const int rl = rb + i * rg;
             if (rl < rows) {  // the same for the whole warp
               const int v = __reduce_add_sync(0xffffffffu, acc[i]);
-              if (lane == 0) part[slice * P.part_stride + rl] = v;
+              if (ks == 1) {  // the row is complete: store it now
+                if (lane == 0) {
+                  const uint32_t y = bf16_bits(epilogue_value(v, r, relu2));
+                  d.Y[r0 + rl] = static_cast<uint16_t>(y);
+                  if (r0 + rl < k_next) wmax = fmaxf(wmax, fabsf(bf16_lo(y)));
+                }
+              } else if (lane == 0) {
+                part[slice * P.part_stride + rl] = v;
+              }
             }
           }
         }
@@ -405,17 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       } else {
         *stop = 1;  // acted on at the next step's first barrier
       }
+      if (lane == 0) red_max[warp] = wmax;
       if (tid == 0) *stop_snap = *stop;
       consumers_sync();
       // ---- warp 0 stores the CTA's outputs (two per 32-bit word), folds
       // their max |y| (over what the next step reads) into the step's max
       // word and counts the CTA in
       if (warp == 0 && !*stop_snap) {
-        const bool last = s + 1 == P.n_steps;
-        const int k_next = last ? 0 : tab[s + 1].K;
-        const bool relu2 = (d.flags & kStepRelu2) != 0;
-        float la = 0.0f;
-        for (int pl = lane; 2 * pl < rows; pl += 32) {
+        float la = lane < kCWarps ? red_max[lane] : 0.0f;
+        for (int pl = lane; ks > 1 && 2 * pl < rows; pl += 32) {
           const bool has_b = 2 * pl + 1 < rows;
           int aa = 0, ab = 0;
           for (int k = 0; k < ks; ++k) {
@@ -435,8 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
         __syncwarp();
         if (lane == 0) {
-          if (!last) P.maxima[static_cast<size_t>(s) * kMaxCtas + blockIdx.x] = la;
-          fence_acq_rel_gpu();  // the warp's stores and the maximum before the count
+          if (!last && (r0 < k_next || blockIdx.x == 0))
+            atomicMax(P.amax + static_cast<size_t>(s) * 16,
+                      (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(la));
+          fence_acq_rel_gpu();  // every warp's stores and the max before the count
           red_release_add(P.arrive + static_cast<size_t>(s) * 32, 1u);
         }
       }
@@ -550,8 +572,8 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   p.epoch = reinterpret_cast<unsigned *>(ws);
   p.arrive = reinterpret_cast<unsigned *>(ws + kChainWorkspaceHeader);
-  p.maxima = reinterpret_cast<float *>(ws + kChainWorkspaceHeader +
-                                      static_cast<size_t>(n_steps) * kChainLine);
+  p.amax = reinterpret_cast<unsigned long long *>(ws + kChainWorkspaceHeader +
+                                                  static_cast<size_t>(n_steps) * kChainLine);
   p.status = ctx.status;
   p.n_steps = n_steps;
   p.ctas = plan.ctas;

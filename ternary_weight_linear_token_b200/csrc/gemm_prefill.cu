@@ -40,6 +40,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "quant_row.cuh"
 
 namespace bitnet {
 namespace {
@@ -51,6 +52,12 @@ constexpr int kEpiWarps = 4;
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
 constexpr int kThreads = 32 * (kEpiWarps + 2);
+// The fused form adds warps that prepare the operands (quantise the token
+// rows, expand the packed weight rows) while the pipeline runs.
+constexpr int kPrepWarps = 6;
+constexpr int kWarpPrep0 = kEpiWarps + 2;
+constexpr int kThreadsFused = 32 * (kEpiWarps + 2 + kPrepWarps);
+constexpr int kReadyStride = 8;  // readiness counters 32 bytes apart
 constexpr int kABytes = BM * BK;
 constexpr int kTmemCols = 2 * BN;
 constexpr int kStoreRows = 32;                    // epilogue staging block: 32 rows
@@ -80,7 +87,153 @@ struct PrefillParams {
   int *status;
   int64_t M, N, K;
   int m_tiles, n_tiles;
+  // the fused form: operands prepared inside the kernel.  ready[] counts the
+  // rows done per block of a tile's token rows (m_tiles of them), then per
+  // 256-row block of weights (n_tiles); a tile's loads wait for both.
+  const void *X;        // raw activations (fp32/bf16), or null: xq is given
+  int x_kind;
+  int8_t *xq;           // where the quantised activations go (TMA source)
+  float *s_out;         // their scales (== s)
+  const uint8_t *packed;
+  int8_t *w8;           // where the expanded weights go (TMA source)
+  int expand;           // 0: w8 already holds them
+  unsigned *ready;
 };
+
+// Rows of token block b (tile_m rows each) and of weight block b (BN rows).
+__host__ __device__ inline int block_rows(int64_t total, int64_t rows_per_block, int b) {
+  const int64_t r = total - static_cast<int64_t>(b) * rows_per_block;
+  return static_cast<int>(r < rows_per_block ? r : rows_per_block);
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait (one thread) until a readiness counter reaches `want`, with
+// acquire semantics; then the async proxy (the TMA) may read what the
+// counted rows' writers stored.  False after recording a timeout.
+__device__ __forceinline__ bool wait_ready(const unsigned *ctr, unsigned want, int *status) {
+  if (ld_acquire_u32(ctr) != want) {
+    const long long t0 = clock64();
+    while (ld_acquire_u32(ctr) != want) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        record_status(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+// The counters of a fused launch: each token block starts at 0 when the
+// kernel quantises (else complete), each weight block at 0 when it expands.
+__global__ void prep_reset_kernel(unsigned *ready, int m_tiles, int n_tiles, int64_t M, int64_t N,
+                                  int tile_m, int quantize, int expand) {
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel may still be reading the counters
+  for (int i = threadIdx.x; i < m_tiles + n_tiles; i += blockDim.x) {
+    unsigned v;
+    if (i < m_tiles)
+      v = quantize ? 0u : static_cast<unsigned>(block_rows(M, tile_m, i));
+    else
+      v = expand ? 0u : static_cast<unsigned>(block_rows(N, BN, i - m_tiles));
+    ready[static_cast<size_t>(i) * kReadyStride] = v;
+  }
+}
+
+// A batch of weight rows expanded by one warp with all of its loads in
+// flight at once (kExpandWordsInFlight packed words per lane), then one
+// proxy fence per lane and one release count per row.
+constexpr int kExpandWordsInFlight = 32;
+template <bool PERM>
+__device__ __forceinline__ void expand_rows_batch(const PrefillParams &p, int64_t n_first,
+                                                  int64_t n_step, int count, int lane) {
+  const int words = static_cast<int>(p.K / 16);
+  const uint32_t *src = reinterpret_cast<const uint32_t *>(p.packed);
+  uint4 *dst = reinterpret_cast<uint4 *>(p.w8);
+  uint32_t v[kExpandWordsInFlight];
+  // flat index i over (row j, word w) of the batch, lane-strided
+  const int total = count * words;
+#pragma unroll
+  for (int k = 0; k < kExpandWordsInFlight; ++k) {
+    const int i = lane + 32 * k;
+    v[k] = 0u;
+    if (i < total) {
+      const int j = i / words, w = i - j * words;
+      v[k] = src[(n_first + n_step * j) * words + w];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kExpandWordsInFlight; ++k) {
+    const int i = lane + 32 * k;
+    if (i < total) {
+      const int j = i / words, w = i - j * words;
+      dst[(n_first + n_step * j) * words + w] = expand_word<PERM>(v[k]);
+    }
+  }
+  fence_proxy_async_global();
+  __syncwarp();
+  if (lane < count)
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(
+                     p.ready + static_cast<size_t>(p.m_tiles + (n_first + n_step * lane) / BN) * kReadyStride)
+                 : "memory");
+}
+
+// One prep warp's share of the operand preparation, in the order the tiles
+// need it (tiles go token block by token block, all weight blocks each):
+// this CTA's rows of the first three token blocks, then its weight rows,
+// then its other token rows.  Row r is this CTA's when r % ctas == cta;
+// warp q of the CTA takes every kPrepWarps-th of those.  After each token
+// row, and after each batch of weight rows, the warp makes its stores
+// visible to the TMA and counts the rows in, with release semantics.
+template <int KIND, bool PERM>
+__device__ __forceinline__ void prep_work(const PrefillParams &p, int tile_m, int cta, int ctas,
+                                          int q, int lane) {
+  const int64_t early = static_cast<int64_t>(tile_m) * 3;
+  const int64_t step = static_cast<int64_t>(ctas) * kPrepWarps;
+  auto tokens = [&](int64_t lo, int64_t hi) {
+    if (p.X == nullptr) return;
+    for (int64_t m = cta + static_cast<int64_t>(ctas) * q; m < hi; m += step) {
+      if (m < lo) continue;
+      quantize_row_warp<KIND, PERM>(p.X, m, p.K, lane, p.xq, p.s_out);
+      fence_proxy_async_global();
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(
+                         p.ready + static_cast<size_t>(m / tile_m) * kReadyStride)
+                     : "memory");
+    }
+  };
+  tokens(0, early < p.M ? early : p.M);
+  if (p.expand) {
+    const int words = static_cast<int>(p.K / 16);
+    int batch = kExpandWordsInFlight * 32 / words;  // rows whose words fit in flight at once
+    if (batch > 32) batch = 32;
+    if (batch >= 1) {
+      for (int64_t n = cta + static_cast<int64_t>(ctas) * q; n < p.N; n += step * batch) {
+        const int64_t left = (p.N - 1 - n) / step + 1;
+        expand_rows_batch<PERM>(p, n, step, static_cast<int>(left < batch ? left : batch), lane);
+      }
+    } else {  // long rows: one at a time
+      for (int64_t n = cta + static_cast<int64_t>(ctas) * q; n < p.N; n += step) {
+        expand_row_warp<PERM>(p.packed, p.w8, n, p.K, lane);
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0)
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(
+                           p.ready + static_cast<size_t>(p.m_tiles + n / BN) * kReadyStride)
+                       : "memory");
+      }
+    }
+  }
+  tokens(early, p.M);
+}
 
 template <int YK, bool RELU2>
 __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64_t n,
@@ -138,8 +291,8 @@ __device__ __forceinline__ void store16(const PrefillParams &p, int64_t m, int64
 
 // PAIR: launched as clusters of two CTAs; the first issues the pair MMAs for
 // both, each loads its own halves of A and B and writes its own 128 rows.
-template <int YK, bool RELU2, bool TMA_Y, bool PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int YK, bool RELU2, bool TMA_Y, bool PAIR, bool FUSED>
+__global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_y, const PrefillParams p) {
@@ -199,6 +352,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = unit; tile < tiles && ok; tile += units) {
         const int32_t m0 = (tile / p.n_tiles) * C::kTileM + static_cast<int32_t>(rank) * BM;
         const int32_t n0 = (tile % p.n_tiles) * BN + static_cast<int32_t>(rank) * C::kBRows;
+        if (FUSED) {  // the tile's token rows and weight rows are prepared
+          const int mb = tile / p.n_tiles, nb = tile % p.n_tiles;
+          ok = wait_ready(p.ready + static_cast<size_t>(mb) * kReadyStride,
+                          static_cast<unsigned>(block_rows(p.M, C::kTileM, mb)), p.status) &&
+               wait_ready(p.ready + static_cast<size_t>(p.m_tiles + nb) * kReadyStride,
+                          static_cast<unsigned>(block_rows(p.N, BN, nb)), p.status);
+          if (!ok) break;
+        }
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % C::kStages;
           if (it >= C::kStages &&
@@ -259,6 +420,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&acc_full[acc]);
       }
     }
+  } else if (FUSED && warp >= kWarpPrep0) {
+    // ---- prep warps: quantise token rows, expand weight rows
+    const int cta = static_cast<int>(blockIdx.x), ctas = static_cast<int>(gridDim.x);
+    const int q = warp - kWarpPrep0;
+    if (p.x_kind == kF32)
+      prep_work<kF32, true>(p, C::kTileM, cta, ctas, q, lane);
+    else if (p.x_kind == kBF16)
+      prep_work<kBF16, true>(p, C::kTileM, cta, ctas, q, lane);
+    else
+      prep_work<kBF16, false>(p, C::kTileM, cta, ctas, q, lane);  // int8 given: expansion only
   } else {
     // ---- epilogue warps 0-3: TMEM lane quadrant = warp
     const int q = warp;
@@ -277,6 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                              static_cast<int64_t>(rank) * BM + q * 32;
       const int64_t m = m_base + lane;
       const int64_t n0 = static_cast<int64_t>(tile % p.n_tiles) * BN;
+      if (FUSED) {  // the scales come from the prep warps (complete once the tile ran)
+        if (lane == 0) (void)ld_acquire_u32(p.ready + static_cast<size_t>(tile / p.n_tiles) * kReadyStride);
+        __syncwarp();
+      }
       const float r = (m < p.M) ? __fdiv_rn(gamma, p.s[m]) : 0.0f;
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(acc * BN) +
                              (static_cast<uint32_t>(q * 32) << 16);
@@ -385,21 +560,22 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int YK, bool RELU2, bool TMA_Y, bool PAIR>
+template <int YK, bool RELU2, bool TMA_Y, bool PAIR, bool FUSED>
 cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
                const PrefillParams &p, const LaunchCtx &ctx) {
   using C = Cfg<PAIR>;
-  auto kern = prefill_kernel<YK, RELU2, TMA_Y, PAIR>;
+  auto kern = prefill_kernel<YK, RELU2, TMA_Y, PAIR, FUSED>;
+  const int threads = FUSED ? kThreadsFused : kThreads;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmemBytes));
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   if (!PAIR) {
     const dim3 grid(static_cast<unsigned>(tiles < ctx.num_sms ? tiles : ctx.num_sms));
-    return launch_k(kern, grid, dim3(kThreads), C::kSmemBytes, ctx, ta, tb, ty, p);
+    return launch_k(kern, grid, dim3(threads), C::kSmemBytes, ctx, ta, tb, ty, p);
   }
-  // as many pairs as the device can hold at once (asked once per device); none: the
-  // caller runs single CTAs
+  // as many pairs as the device can hold at once (asked once per device and
+  // form); none: the caller runs single CTAs
   static std::atomic<int> resident[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
@@ -407,7 +583,7 @@ cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &
   if (most == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * (ctx.num_sms / 2)));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -428,21 +604,33 @@ cudaError_t go(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &
   int64_t pairs = ctx.num_sms / 2;
   if (pairs > most) pairs = most;
   const dim3 grid(static_cast<unsigned>(2 * (tiles < pairs ? tiles : pairs)));
-  return launch_k_cluster(kern, grid, dim3(kThreads), C::kSmemBytes, 2u, ctx, ta, tb, ty, p);
+  return launch_k_cluster(kern, grid, dim3(threads), C::kSmemBytes, 2u, ctx, ta, tb, ty, p);
+}
+
+template <bool PAIR, bool FUSED>
+cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, bool tma_y,
+                 const PrefillParams &p, int y_kind, bool relu2, const LaunchCtx &ctx) {
+  if (y_kind == kI32) return go<kI32, false, false, PAIR, FUSED>(ta, tb, ty, p, ctx);
+  if (y_kind == kF32)
+    return relu2 ? go<kF32, true, false, PAIR, FUSED>(ta, tb, ty, p, ctx)
+                 : go<kF32, false, false, PAIR, FUSED>(ta, tb, ty, p, ctx);
+  if (tma_y)
+    return relu2 ? go<kBF16, true, true, PAIR, FUSED>(ta, tb, ty, p, ctx)
+                 : go<kBF16, false, true, PAIR, FUSED>(ta, tb, ty, p, ctx);
+  return relu2 ? go<kBF16, true, false, PAIR, FUSED>(ta, tb, ty, p, ctx)
+               : go<kBF16, false, false, PAIR, FUSED>(ta, tb, ty, p, ctx);
 }
 
 template <bool PAIR>
-cudaError_t go_y(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, bool tma_y,
+cudaError_t go_f(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, bool tma_y,
                  const PrefillParams &p, int y_kind, bool relu2, const LaunchCtx &ctx) {
-  if (y_kind == kI32) return go<kI32, false, false, PAIR>(ta, tb, ty, p, ctx);
-  if (y_kind == kF32)
-    return relu2 ? go<kF32, true, false, PAIR>(ta, tb, ty, p, ctx)
-                 : go<kF32, false, false, PAIR>(ta, tb, ty, p, ctx);
-  if (tma_y)
-    return relu2 ? go<kBF16, true, true, PAIR>(ta, tb, ty, p, ctx)
-                 : go<kBF16, false, true, PAIR>(ta, tb, ty, p, ctx);
-  return relu2 ? go<kBF16, true, false, PAIR>(ta, tb, ty, p, ctx)
-               : go<kBF16, false, false, PAIR>(ta, tb, ty, p, ctx);
+  if (p.ready == nullptr) return go_y<PAIR, false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+  // the counters first: a one-CTA kernel, launched as the fused kernel's predecessor
+  const bool quantize = p.X != nullptr;
+  const cudaError_t e = launch_k(prep_reset_kernel, dim3(1), dim3(256), 0, ctx, p.ready, p.m_tiles,
+                                 p.n_tiles, p.M, p.N, Cfg<PAIR>::kTileM, quantize ? 1 : 0, p.expand);
+  if (e != cudaSuccess) return e;
+  return go_y<PAIR, true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
 }
 
 }  // namespace
@@ -457,9 +645,13 @@ bool prefill_supported(int64_t M, int64_t N, int64_t K) {
 
 size_t prefill_weight_bytes(int64_t N, int64_t K) { return static_cast<size_t>(N) * K; }
 
+size_t prefill_ready_bytes(int64_t M, int64_t N) {
+  return static_cast<size_t>(4 * kReadyStride) * static_cast<size_t>(ceil_div(M, BM) + ceil_div(N, BN));
+}
+
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, const LaunchCtx &ctx) {
+                           void *Y, int y_kind, const LaunchCtx &ctx, const PrefillPrep *prep) {
   PrefillParams p;
   p.s = s;
   p.gamma = gamma;
@@ -469,6 +661,21 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
   p.N = N;
   p.K = K;
   p.n_tiles = static_cast<int>(ceil_div(N, BN));
+  p.X = nullptr;
+  p.x_kind = kI8;
+  p.xq = const_cast<int8_t *>(xq);
+  p.s_out = const_cast<float *>(s);
+  p.packed = nullptr;
+  p.w8 = const_cast<int8_t *>(w8);
+  p.expand = 0;
+  p.ready = nullptr;
+  if (prep != nullptr && (prep->X != nullptr || prep->packed != nullptr)) {
+    p.X = prep->X;
+    p.x_kind = prep->X != nullptr ? prep->x_kind : kI8;
+    p.packed = prep->packed;
+    p.expand = prep->packed != nullptr ? 1 : 0;
+    p.ready = prep->ready;
+  }
   CUtensorMap ta, tb, ty;
   if (!make_map_2d(&ta, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
                    static_cast<uint64_t>(K), BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -485,14 +692,14 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                      static_cast<uint64_t>(K), BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     p.m_tiles = static_cast<int>(ceil_div(M, 2 * BM));
-    const cudaError_t e = go_y<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+    const cudaError_t e = go_f<true>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
     if (e != cudaErrorInvalidClusterSize) return e;  // else: no pair fits, single CTAs
   }
   if (!make_map_2d(&tb, w8, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                    static_cast<uint64_t>(K), BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   p.m_tiles = static_cast<int>(ceil_div(M, BM));
-  return go_y<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
+  return go_f<false>(ta, tb, ty, tma_y, p, y_kind, relu2, ctx);
 }
 
 }  // namespace bitnet

@@ -81,9 +81,21 @@ cudaError_t launch_generic(const int8_t *xq, const float *s, const uint8_t *pack
 bool prefill_shape_ok(int64_t M, int64_t N, int64_t K);
 bool prefill_supported(int64_t M, int64_t N, int64_t K);
 size_t prefill_weight_bytes(int64_t N, int64_t K);
+// Operands the tensor-core kernel prepares itself while it runs (the fused
+// form): the raw activations X (quantised, in xq's K order, into xq and s),
+// and/or the packed weights (expanded into w8).  `ready` is scratch of
+// prefill_ready_bytes(M, N) bytes for its per-block readiness counters.
+struct PrefillPrep {
+  const void *X = nullptr;        // null: xq and s are given
+  int x_kind = 0;
+  const uint8_t *packed = nullptr;  // null: w8 is given
+  unsigned *ready = nullptr;
+};
+size_t prefill_ready_bytes(int64_t M, int64_t N);
 cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            const float *gamma, int64_t M, int64_t N, int64_t K, bool relu2,
-                           void *Y, int y_kind, const LaunchCtx &ctx);
+                           void *Y, int y_kind, const LaunchCtx &ctx,
+                           const PrefillPrep *prep = nullptr);
 
 // chain.cu: persistent M = 1 chain of BitLinear projections (one
 // cooperative launch).  Step flags mirror BITNET_STEP_*.
@@ -93,11 +105,9 @@ constexpr int kStepNormIn = 2;
 constexpr size_t kChainWorkspaceHeader = 256;  // the launch counter at byte 0
 constexpr int kChainMaxCtas = 256;              // CTAs of one chain launch, at most
 // After the header, one 128-byte line per step holding its arrival counter,
-// then per step kChainMaxCtas floats: each CTA's max |y| of the step.
+// then one per step holding its tagged max |y| word.
 constexpr size_t kChainLine = 128;
-inline size_t chain_sync_bytes(int n_steps) {
-  return (kChainLine + 4 * static_cast<size_t>(kChainMaxCtas)) * static_cast<size_t>(n_steps);
-}
+inline size_t chain_sync_bytes(int n_steps) { return 2 * kChainLine * static_cast<size_t>(n_steps); }
 struct ChainStep {
   const uint8_t *packed;
   const float *gamma;

@@ -70,7 +70,7 @@ def test_matmul_rejects_bad_arguments(tw):
     assert mm(tw, yd=2) == tw.ERR_INVALID_ARG            # int8 output
     assert mm(tw, epi=2) == tw.ERR_INVALID_ARG
     assert mm(tw, yd=3, epi=1) == tw.ERR_INVALID_ARG     # raw int32 with ReLU^2
-    assert mm(tw, flags=8) == tw.ERR_INVALID_ARG         # unknown flag bit
+    assert mm(tw, flags=16) == tw.ERR_INVALID_ARG        # unknown flag bit
     assert mm(tw, M=-1) == tw.ERR_INVALID_ARG
     assert mm(tw, K=0) == tw.ERR_INVALID_ARG
     assert mm(tw, K=40) == tw.ERR_UNSUPPORTED_SHAPE      # not a multiple of 16
@@ -101,10 +101,13 @@ def test_workspace_sizes(tw):
     assert f(8, 6912, 2560, tw.I8) == 0                   # xq given
     assert f(32, 2560, 6912, tw.BF16) == 32 * 6912 + 256
     assert f(16, 2560, 6912, tw.I8) == 0            # xq given, mma.sync path
-    # tensor-core path: xq and s (float input only), then the int8 weights
-    assert f(4096, 6912, 2560, tw.I8) == 6912 * 2560
-    assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4 + 6912 * 2560
-    assert f(33, 7, 64, tw.F32) == 2304 + 256 + 512       # each part rounded up to 256
+    # tensor-core path: xq and s (float input only), then the int8 weights,
+    # then 32 bytes of readiness counter per 128 tokens and per 256 features
+    ready = (4096 // 128 + (6912 + 255) // 256) * 32   # 1888 -> 2048
+    assert f(4096, 6912, 2560, tw.I8) == 6912 * 2560 + 2048
+    assert f(4096, 6912, 2560, tw.BF16) == 4096 * 2560 + 4096 * 4 + 6912 * 2560 + 2048
+    assert ready <= 2048
+    assert f(33, 7, 64, tw.F32) == 2304 + 256 + 512 + 256  # each part rounded up to 256
     assert f(40, 33, 80, tw.I8) == 0                # K % 64 != 0: generic kernel
     assert f(5, 64, 48, tw.F32) == 0                # M <= 8 and K % 64 != 0: fused kernel
     assert f(9, 64, 48, tw.F32) == 512 + 256        # generic path (M > 8, K % 64 != 0)
@@ -175,11 +178,11 @@ def test_decode_chain_workspace_size(tw):
     f = tw.lib.bitnet_decode_chain_workspace_size
     layer = [(3840, 2560), (2560, 2560), (6912, 2560), (2560, 6912)]
     # 256-byte header (the launch counter); then one 128-byte line per step
-    # for its arrival counter, then per step 256 floats (each CTA's max |y|)
-    assert f(chain(tw, layer), 4) == (256 + 4 * 1152 + 255) // 256 * 256
-    assert f(chain(tw, [(333, 64)]), 1) == 1536      # 256 + 1152 = 1408, rounded up
+    # for its arrival counter and one for its tagged max |y| word
+    assert f(chain(tw, layer), 4) == 256 + 4 * 256
+    assert f(chain(tw, [(333, 64)]), 1) == 512
     assert f(chain(tw, [(64, 40)]), 1) == 0          # invalid descriptors
-    assert f(chain(tw, layer * 30), 120) == 256 + 120 * 1152
+    assert f(chain(tw, layer * 30), 120) == 256 + 120 * 256
 
 
 def test_rms_norm_matmul_rejects_bad_arguments(tw):
@@ -245,7 +248,7 @@ def test_noalloc_checks_arguments_before_its_size_limit(tw):
     assert call(xd=3) == tw.ERR_INVALID_ARG
     assert call(xd=7) == tw.ERR_INVALID_ARG
     assert call(yd=2) == tw.ERR_INVALID_ARG
-    assert call(flags=8) == tw.ERR_INVALID_ARG
+    assert call(flags=16) == tw.ERR_INVALID_ARG
     assert call(M=1 << 40) == tw.ERR_INVALID_ARG
     assert call(K=40) == tw.ERR_UNSUPPORTED_SHAPE
     assert call(X=MIS) == tw.ERR_MISALIGNED

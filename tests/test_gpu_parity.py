@@ -173,6 +173,42 @@ def test_matmul_parity(tw, M, N, K, xdtype):
     assert all(exact.values()), f"within tolerance but not bit-identical: {exact}"
 
 
+PREP_SHAPES = [(33, 300, 192), (128, 256, 128), (129, 257, 2624), (300, 600, 2560),
+               (256, 520, 64), (1000, 512, 2560), (640, 1100, 384), (130, 70, 208)]
+
+
+@pytest.mark.parametrize("M,N,K", [sh for sh in PREP_SHAPES if sh[2] % 64 == 0])
+@pytest.mark.parametrize("xdtype", ["f32", "bf16", "i8"])
+def test_prep_in_kernel_parity(tw, M, N, K, xdtype):
+    """The tensor-core path with its operands prepared inside the kernel
+    (BITNET_FLAG_PREP_IN_KERNEL): single CTAs and CTA pairs, ragged M, N and
+    K, every input dtype; int32 accumulators and outputs bit-exact."""
+    rng = np.random.default_rng(M * 7907 + N * 13 + K)
+    W = synth.latent_weights(rng, N, K)
+    x = rng.standard_t(3, (M, K)).astype(np.float32)
+    packed_d, gamma_d, packed_o, gamma_o = quantize_weights_both(W)
+    if xdtype == "i8":
+        xq_o, s_o = ref.quantize_act(x)
+        Xd, sd = torch.from_numpy(xq_o).to(DEV), torch.from_numpy(s_o).to(DEV)
+    else:
+        Xd, xexact = as_x(x, xdtype)
+        sd = None
+        xq_o, s_o = ref.quantize_act(xexact)
+    assert tw.bitnet_w158a8_matmul_path(M, N, K, Xd.dtype) == tw.PATH_TENSOR_CORE
+    acc_o = ref.matmul_acc(xq_o, packed_o, N, K)
+    for out_dtype, relu2 in ((torch.int32, False), (torch.bfloat16, True), (torch.float32, False)):
+        Y = tw.bitnet_w158a8_matmul(Xd, packed_d, gamma_d, s=sd, relu2=relu2, out_dtype=out_dtype,
+                                    prep_in_kernel=True)
+        torch.cuda.synchronize()
+        if out_dtype == torch.int32:
+            assert np.array_equal(np_of(Y), acc_o)
+        elif out_dtype == torch.float32:
+            assert np.array_equal(np_of(Y), ref.epilogue(acc_o, s_o, gamma_o, relu2))
+        else:
+            assert np.array_equal(bf16_bits_of(Y), ref.to_bf16(ref.epilogue(acc_o, s_o, gamma_o, relu2)))
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
 # the table-lookup comparison kernel: 1..8 tokens, several CTAs' rows, K
 # ragged against the 32-lane word loop, K of the down projection (one
 # token's tables per batch), more tokens than fit in one table batch
@@ -333,6 +369,13 @@ def test_prefill_workload_full_size(tw):
                                  weights_expanded=True)
     torch.cuda.synchronize()
     assert np.array_equal(bf16_bits_of(Y2), want)
+    # the tensor-core kernel preparing its own operands (quantiser and
+    # expansion inside the kernel, BITNET_FLAG_PREP_IN_KERNEL): same outputs
+    ws2 = torch.empty(need, dtype=torch.uint8, device=DEV)
+    Y4 = tw.bitnet_w158a8_matmul(Xd, pd, gd, workspace=ws2, weights_static=True,
+                                 prep_in_kernel=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits_of(Y4), want)
     # int8 activations from the caller (natural K order, its own expansion),
     # then again with that expansion kept
     xq, sq = tw.bitnet_quantize_act(Xd)
