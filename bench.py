@@ -340,7 +340,8 @@ def make_prefill(tw, torch, dev, l2_bytes, prep_in_kernel=False):
                            "int8 scratch runs in the same launch) + tcgen05 kernel")},
         kernel_key="prefill_tcgen05_M4096_K2560_N6912",
         kernel_files=["ternary_weight_linear_token_b200/csrc/gemm_prefill.cu",
-                      "ternary_weight_linear_token_b200/csrc/common.cuh"],
+                      "ternary_weight_linear_token_b200/csrc/common.cuh",
+                      "ternary_weight_linear_token_b200/csrc/quant_row.cuh"],
         e2e_inputs=lambda: (d["x_bits"].view(np.int16), 2 * M * K, 2 * M * N),
     )
 
