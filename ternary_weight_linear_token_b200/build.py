@@ -27,7 +27,7 @@ LIB = os.path.join(PKG, "libbitnet158.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--fmad=false", "-Xcompiler", "-fPIC",
-              "-Xcompiler", "-Wall", "-Xlinker", "--exclude-libs,ALL"]
+              "-Xcompiler", "-Wall"]
 
 
 def sources() -> list[str]:
@@ -51,10 +51,26 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+    """Compile every source to its own object (in parallel, under _build/ beside
+    the sources), then link the shared library."""
     if not force and not _stale():
         return LIB
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-shared", *sources(),
-           "-o", LIB + ".tmp"]
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [*ARCH, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE]
+
+    def compile_one(src: str) -> str:
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *flags, "-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.run(cmd, check=True, cwd=PKG)
+        return obj
+
+    with ThreadPoolExecutor(max_workers=max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(compile_one, sources()))
+    cmd = [nvcc(), *ARCH, "-Xlinker", "--exclude-libs,ALL", "-shared", *objs, "-o", LIB + ".tmp"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True, cwd=PKG)

@@ -28,12 +28,10 @@
 //   * Per link, each CTA quantises the whole input to int8 exactly as
 //     bitnet_quantize_act does and computes its balanced range of output
 //     features with the byte-permute unpack and dp4a, in the same int32
-//     arithmetic and with the same epilogue as bitnet_w158a8_matmul.  The
-//     16 consumer warps form a grid, chosen per step: ks slices of K times
-//     16 / ks groups of rows, the split that gives the busiest warp the
-//     fewest dot products; a lane loads each of its activation chunks once
-//     per pass of up to 4 rows.  With one slice a warp finishes its rows
-//     itself; otherwise warp 0 adds the slices' partial sums.
+//     arithmetic and with the same epilogue as bitnet_w158a8_matmul.  Warp
+//     w takes rows w, w + 16, ... of the CTA's range, up to 4 at a time: a
+//     lane loads each of its activation chunks once per pass and uses it for
+//     all of the pass's rows, and stores each row as soon as it is done.
 //   * The counters only grow: launch T (T = the launch counter kept in the
 //     workspace, plus one) waits for T * ctas arrivals; CTA 0 advances the
 //     launch counter once all CTAs have passed the last step, so graph
@@ -82,7 +80,7 @@ struct ChainP {
   unsigned *arrive;           // [n_steps], one per 128-byte line
   unsigned long long *amax;   // [n_steps], one per 128-byte line: tag << 32 | max |y| bits
   int *status;
-  int n_steps, ctas, slots, slot_bytes, xq_bytes, part_bytes, part_stride, y_norm_n;
+  int n_steps, ctas, slots, slot_bytes, xq_bytes, y_norm_n;
   StepP steps[kChainMaxSteps];
 };
 
@@ -186,24 +184,6 @@ __device__ __forceinline__ bool wait_or_stop(uint64_t *bar, uint32_t parity,
   }
 }
 
-// K slices of the consumer warp grid for `rows` rows of `words` packed
-// words: the power of two ks (1..16; 16 / ks groups of rows) that gives the
-// busiest warp the fewest dot products of a packed word, ceil(rows / rg)
-// rows times ceil(words / (32 ks)) words per lane; the fewest slices among
-// equals.
-__device__ __forceinline__ int k_slices(int rows, int words) {
-  int best = 1, cost = 0x7fffffff;
-  for (int ks = 1; ks <= kCWarps; ks <<= 1) {
-    const int rg = kCWarps / ks;
-    const int c = ((rows + rg - 1) / rg) * ((words + 32 * ks - 1) / (32 * ks));
-    if (c < cost) {
-      cost = c;
-      best = ks;
-    }
-  }
-  return best;
-}
-
 __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constant__ ChainP P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);                // [kMaxSlots]
@@ -221,8 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   float *gam = reinterpret_cast<float *>(smem + kHeader + align128(P.n_steps * 48));
   int2 *rr = reinterpret_cast<int2 *>(smem + kHeader + align128(P.n_steps * 48) +
                                       align128(P.n_steps * 4));       // this CTA's rows
-  int *part = reinterpret_cast<int *>(smem + kHeader + table_bytes(P.n_steps));  // [16][part_stride]
-  uint8_t *xq = smem + kHeader + table_bytes(P.n_steps) + P.part_bytes;    // [xq_bytes]
+  uint8_t *xq = smem + kHeader + table_bytes(P.n_steps);                  // [xq_bytes]
   uint8_t *slots = xq + P.xq_bytes;                                   // [slots][slot_bytes]
   const uint4 *xq4 = reinterpret_cast<const uint4 *>(xq);
 
@@ -381,7 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       const bool have_w = __all_sync(0xffffffffu, mbar_wait(full + slot, phase, P.status));
       const int r0 = rr[s].x, rows = rr[s].y - r0;
       const int words = d.K >> 4;  // packed 32-bit words per row
-      const int ks = k_slices(rows, words), rg = kCWarps / ks;
       const bool last = s + 1 == P.n_steps;
       const int k_next = last ? 0 : tab[s + 1].K;
       const bool relu2 = (d.flags & kStepRelu2) != 0;
@@ -390,34 +368,27 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         consumed = s + 1;
         const uint32_t *wsl =
             reinterpret_cast<const uint32_t *>(slots + static_cast<size_t>(slot) * P.slot_bytes);
-        // warp (slice, group): words [w0, w1) of rows group, group + rg, ...
-        const int slice = warp / rg, group = warp - slice * rg;
-        const int w0 = slice * words / ks, w1 = (slice + 1) * words / ks;
-        for (int rb = group; rb < rows; rb += rg * kRowsPerPass) {
+        for (int rb = warp; rb < rows; rb += kCWarps * kRowsPerPass) {
           int acc[kRowsPerPass];
 #pragma unroll
           for (int i = 0; i < kRowsPerPass; ++i) acc[i] = 0;
-          for (int w = w0 + lane; w < w1; w += 32) {
+          for (int w = lane; w < words; w += 32) {
             const uint4 x = xq4[w];
 #pragma unroll
             for (int i = 0; i < kRowsPerPass; ++i) {
-              const int rl = rb + i * rg;
+              const int rl = rb + i * kCWarps;
               if (rl < rows) acc[i] = dot_word(unpack_word(wsl[static_cast<size_t>(rl) * words + w]), x, acc[i]);
             }
           }
 #pragma unroll
           for (int i = 0; i < kRowsPerPass; ++i) {
-            const int rl = rb + i * rg;
+            const int rl = rb + i * kCWarps;
             if (rl < rows) {  // the same for the whole warp
               const int v = __reduce_add_sync(0xffffffffu, acc[i]);
-              if (ks == 1) {  // the row is complete: store it now
-                if (lane == 0) {
-                  const uint32_t y = bf16_bits(epilogue_value(v, r, relu2));
-                  d.Y[r0 + rl] = static_cast<uint16_t>(y);
-                  if (r0 + rl < k_next) wmax = fmaxf(wmax, fabsf(bf16_lo(y)));
-                }
-              } else if (lane == 0) {
-                part[slice * P.part_stride + rl] = v;
+              if (lane == 0) {  // the row is complete: store it now
+                const uint32_t y = bf16_bits(epilogue_value(v, r, relu2));
+                d.Y[r0 + rl] = static_cast<uint16_t>(y);
+                if (r0 + rl < k_next) wmax = fmaxf(wmax, fabsf(bf16_lo(y)));
               }
             }
           }
@@ -435,29 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       // word and counts the CTA in
       if (warp == 0 && !*stop_snap) {
         float la = lane < kCWarps ? red_max[lane] : 0.0f;
-        for (int pl = lane; ks > 1 && 2 * pl < rows; pl += 32) {
-          const bool has_b = 2 * pl + 1 < rows;
-          int aa = 0, ab = 0;
-          for (int k = 0; k < ks; ++k) {
-            aa += part[k * P.part_stride + 2 * pl];
-            if (has_b) ab += part[k * P.part_stride + 2 * pl + 1];
-          }
-          const uint32_t ya = bf16_bits(epilogue_value(aa, r, relu2));
-          const uint32_t yb = has_b ? bf16_bits(epilogue_value(ab, r, relu2)) : 0u;
-          if (has_b)
-            *reinterpret_cast<uint32_t *>(d.Y + r0 + 2 * pl) = (yb << 16) | ya;
-          else
-            d.Y[r0 + 2 * pl] = static_cast<uint16_t>(ya);
-          const int g = r0 + 2 * pl;
-          if (g < k_next) la = fmaxf(la, fabsf(bf16_lo(ya)));
-          if (has_b && g + 1 < k_next) la = fmaxf(la, fabsf(bf16_lo(yb)));
-        }
         la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
         __syncwarp();
         if (lane == 0) {
-          if (!last && (r0 < k_next || blockIdx.x == 0))
-            atomicMax(P.amax + static_cast<size_t>(s) * 16,
-                      (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(la));
+          if (!last && (r0 < k_next || blockIdx.x == 0))  // no value returned: nothing to wait for
+            asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(
+                             P.amax + static_cast<size_t>(s) * 16),
+                         "l"((static_cast<unsigned long long>(tag) << 32) | __float_as_uint(la))
+                         : "memory");
           fence_acq_rel_gpu();  // every warp's stores and the max before the count
           red_release_add(P.arrive + static_cast<size_t>(s) * 32, 1u);
         }
@@ -533,20 +489,18 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
 
 bool chain_plan(const ChainStep *steps, int n_steps, int num_sms, ChainPlan *plan) {
   const int ctas = num_sms < kMaxCtas ? num_sms : kMaxCtas;
-  int64_t slot_bytes = 0, max_rows = 0;
+  int64_t slot_bytes = 0;
   int max_k = 0;
   for (int s = 0; s < n_steps; ++s) {
     const int64_t pairs = (steps[s].N + 1) / 2;
     const int64_t rows = 2 * ((pairs + ctas - 1) / ctas);
     const int64_t b = rows * (steps[s].K / 4);
     if (b > slot_bytes) slot_bytes = b;
-    if (rows > max_rows) max_rows = rows;
     if (steps[s].K > max_k) max_k = static_cast<int>(steps[s].K);
   }
   slot_bytes = (slot_bytes + 127) / 128 * 128;
-  const int64_t part_bytes = (static_cast<int64_t>(kCWarps) * max_rows * 4 + 127) / 128 * 128;
   const int xq_bytes = (max_k + 127) / 128 * 128;
-  const int64_t room = kSmemLimit - kHeader - table_bytes(n_steps) - part_bytes - xq_bytes;
+  const int64_t room = kSmemLimit - kHeader - table_bytes(n_steps) - xq_bytes;
   int64_t slots = slot_bytes > 0 ? room / slot_bytes : kMaxSlots;
   if (slots > kMaxSlots) slots = kMaxSlots;
   if (slots < 2) return false;
@@ -554,9 +508,7 @@ bool chain_plan(const ChainStep *steps, int n_steps, int num_sms, ChainPlan *pla
   plan->slots = static_cast<int>(slots);
   plan->slot_bytes = static_cast<int>(slot_bytes);
   plan->xq_bytes = xq_bytes;
-  plan->part_bytes = static_cast<int>(part_bytes);
-  plan->part_stride = static_cast<int>(max_rows);
-  plan->smem = static_cast<size_t>(kHeader) + table_bytes(n_steps) + part_bytes + xq_bytes +
+  plan->smem = static_cast<size_t>(kHeader) + table_bytes(n_steps) + xq_bytes +
                static_cast<size_t>(slots) * slot_bytes;
   return true;
 }
@@ -580,8 +532,6 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
   p.slots = plan.slots;
   p.slot_bytes = plan.slot_bytes;
   p.xq_bytes = plan.xq_bytes;
-  p.part_bytes = plan.part_bytes;
-  p.part_stride = plan.part_stride;
   p.y_norm_n = static_cast<int>(y_norm_n);
   for (int s = 0; s < n_steps; ++s) {
     StepP &d = p.steps[s];

@@ -117,7 +117,7 @@ struct ChainStep {
   void *Xn;
 };
 struct ChainPlan {
-  int ctas, slots, slot_bytes, xq_bytes, part_bytes, part_stride;
+  int ctas, slots, slot_bytes, xq_bytes;
   size_t smem;
 };
 int chain_max_k();
