@@ -201,6 +201,32 @@ bitnet_status bitnet_w158a8_matmul(const void *X, bitnet_dtype x_dtype, const fl
                                    uint32_t flags, bitnet_stream_t stream);
 
 /* ----------------------------------------------------------------------
+ * bitnet_w158a8_matmul from host memory to host memory, in one call: the
+ * activations are copied from X_host to the caller's device buffer X_dev,
+ * the product runs on the device (exactly bitnet_w158a8_matmul with X_dev,
+ * same results), the output is copied from the caller's device buffer Y_dev
+ * to Y_host, and the call returns once Y_host holds it (it synchronises
+ * `stream`).  For a caller whose activations and results live on the host:
+ * one C call per forward instead of a copy, a launch, a copy and a wait.
+ *   X_host   [M][K] fp32 or bf16 (x_dtype), host memory; page-locked
+ *            (cudaHostAlloc / cudaHostRegister) for the copy to be
+ *            asynchronous, else it is staged by the driver.
+ *   Y_host   [M][N] of y_dtype, host memory (page-locked likewise).
+ *   X_dev, Y_dev  device buffers of those sizes, 16-byte aligned.
+ * Everything else as bitnet_w158a8_matmul (int8 input is not accepted here:
+ * its scales would need a copy of their own).  Errors: the argument checks
+ * of bitnet_w158a8_matmul on X_dev and Y_dev, BITNET_ERR_INVALID_ARG for a
+ * null host pointer, BITNET_ERR_CUDA when a copy or the synchronisation
+ * fails.
+ * ---------------------------------------------------------------------- */
+bitnet_status bitnet_w158a8_matmul_host(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                                        const uint8_t *packed, const float *gamma, int64_t M,
+                                        int64_t N, int64_t K, bitnet_epilogue epi, void *Y_dev,
+                                        void *Y_host, bitnet_dtype y_dtype, void *workspace,
+                                        size_t workspace_bytes, uint32_t flags,
+                                        bitnet_stream_t stream);
+
+/* ----------------------------------------------------------------------
  * Which kernel path bitnet_w158a8_matmul takes for these sizes on the
  * current device (the paths are listed in the comment above).  Pure host
  * logic, except that the tensor-core path also needs the driver's

@@ -56,6 +56,8 @@ _SIGS = {
     "bitnet_quantize_act": ([_P, _ST, _I64, _I64, _P, _P, _P], _ST),
     "bitnet_w158a8_matmul_workspace_size": ([_I64, _I64, _I64, _ST], _SZ),
     "bitnet_w158a8_matmul_path": ([_I64, _I64, _I64, _ST], _ST),
+    "bitnet_w158a8_matmul_host": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _P, _ST, _P, _SZ,
+                                   C.c_uint32, _P], _ST),
     "bitnet_w158a8_matmul": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST, _P, _SZ,
                               C.c_uint32, _P], _ST),
     "bitnet_rms_norm": ([_P, _ST, _I64, _I64, _P, _ST, _P], _ST),
@@ -223,6 +225,38 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
                                   _stream(stream))
     _check(st, "bitnet_w158a8_matmul")
     return Y
+
+
+def bitnet_w158a8_matmul_host(X_host: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                              X_dev: torch.Tensor, Y_dev: torch.Tensor, Y_host: torch.Tensor,
+                              relu2: bool = False, workspace: torch.Tensor | None = None,
+                              weights_static: bool = False, stream=None) -> torch.Tensor:
+    """Y_host = BitLinear(X_host) in one C call: X_host (CPU, fp32/bf16, best
+    pinned) is copied to X_dev, the product writes Y_dev, which is copied to
+    Y_host (CPU, pinned); returns once Y_host holds the result."""
+    if X_host.is_cuda or Y_host.is_cuda:
+        raise ValueError("X_host and Y_host must be host (CPU) tensors")
+    if not (X_host.is_contiguous() and Y_host.is_contiguous()):
+        raise ValueError("X_host and Y_host must be contiguous")
+    _dev(X_dev, "X_dev", (X_host.dtype,))
+    _dev(Y_dev, "Y_dev", (Y_host.dtype,))
+    _dev(packed, "packed", (torch.uint8,))
+    _dev(gamma, "gamma", (torch.float32,))
+    M, K = X_host.shape
+    N = packed.shape[0]
+    if X_dev.shape != X_host.shape or Y_dev.shape != Y_host.shape or Y_host.shape != (M, N):
+        raise ValueError("X_dev/Y_dev must match the shapes of X_host [M, K] and Y_host [M, N]")
+    need = bitnet_w158a8_matmul_workspace_size(M, N, K, X_host.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X_dev.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.bitnet_w158a8_matmul_host(_ptr(X_host), _DTYPE[X_host.dtype], _ptr(X_dev), _ptr(packed),
+                                       _ptr(gamma), M, N, K, EPI_RELU2 if relu2 else EPI_NONE,
+                                       _ptr(Y_dev), _ptr(Y_host), _DTYPE[Y_host.dtype],
+                                       _ptr(workspace), ws_bytes,
+                                       FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
+    _check(st, "bitnet_w158a8_matmul_host")
+    return Y_host
 
 
 def bitnet_rms_norm_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,

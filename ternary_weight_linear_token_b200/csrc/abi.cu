@@ -346,6 +346,38 @@ size_t bitnet_w158a8_matmul_workspace_size(int64_t M, int64_t N, int64_t K, bitn
   return matmul_workspace(M, N, K, x_dtype);
 }
 
+bitnet_status bitnet_w158a8_matmul_host(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                                        const uint8_t *packed, const float *gamma, int64_t M,
+                                        int64_t N, int64_t K, bitnet_epilogue epi, void *Y_dev,
+                                        void *Y_host, bitnet_dtype y_dtype, void *workspace,
+                                        size_t workspace_bytes, uint32_t flags,
+                                        bitnet_stream_t stream) {
+  if (x_dtype == BITNET_I8) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_matmul(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, epi, Y_dev,
+                                      y_dtype, workspace, workspace_bytes, flags, false))
+    return st;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (X_host == nullptr || Y_host == nullptr) return BITNET_ERR_INVALID_ARG;
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  const size_t x_bytes = static_cast<size_t>(M) * K * elem_size(x_dtype);
+  const size_t y_bytes = static_cast<size_t>(M) * N * elem_size(y_dtype);
+  if (cudaMemcpyAsync(X_dev, X_host, x_bytes, cudaMemcpyHostToDevice, ctx.stream) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  const bool relu2 = epi == BITNET_EPI_RELU2, wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
+  const bitnet_status st =
+      (flags & BITNET_FLAG_TABLE_LOOKUP) != 0
+          ? from_cuda(launch_lut(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y_dev,
+                                 y_dtype, wstatic, ctx))
+          : run_matmul(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y_dev, y_dtype,
+                       workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0,
+                       (flags & BITNET_FLAG_PREP_IN_KERNEL) != 0, ctx);
+  if (st != BITNET_OK) return st;
+  if (cudaMemcpyAsync(Y_host, Y_dev, y_bytes, cudaMemcpyDeviceToHost, ctx.stream) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  return cudaStreamSynchronize(ctx.stream) == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
 bitnet_path bitnet_w158a8_matmul_path(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16 && x_dtype != BITNET_I8)
     return BITNET_PATH_NONE;

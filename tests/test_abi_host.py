@@ -254,3 +254,22 @@ def test_noalloc_checks_arguments_before_its_size_limit(tw):
     assert call(X=MIS) == tw.ERR_MISALIGNED
     assert call(M=8192) == tw.ERR_WORKSPACE               # (8192 + 6912) * 2560 > 32 MiB
     assert call(M=0) == tw.OK
+
+
+def test_host_entry_point_checks(tw):
+    """The host-to-host entry point: the matmul's checks on the device
+    buffers, host pointers required, no int8 input; all before any CUDA call."""
+    f = tw.lib.bitnet_w158a8_matmul_host
+    H = C.c_void_p(0x7000000)
+
+    def call(Xh=H, xd=1, Xd=A, M=1, N=8, K=64, Yd=Cc, Yh=H, yd=1, flags=0):
+        return f(Xh, xd, Xd, B, G, M, N, K, 0, Yd, Yh, yd, None, 0, flags, None)
+
+    assert call(Xh=None) == tw.ERR_INVALID_ARG
+    assert call(Yh=None) == tw.ERR_INVALID_ARG
+    assert call(xd=2) == tw.ERR_INVALID_ARG      # int8 input: its scales would need a copy
+    assert call(Xd=MIS) == tw.ERR_MISALIGNED
+    assert call(K=40) == tw.ERR_UNSUPPORTED_SHAPE
+    assert call(flags=16) == tw.ERR_INVALID_ARG
+    assert call(M=4096, N=6912, K=2560) == tw.ERR_WORKSPACE
+    assert call(M=0) == tw.OK

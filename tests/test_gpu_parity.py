@@ -540,6 +540,35 @@ def test_rms_norm_matmul(tw, M, N, K, dt, relu2):
     assert tw.bitnet_get_device_status() == tw.OK
 
 
+@pytest.mark.parametrize("M,N,K,dt", [(1, 2560, 2560, "bf16"), (8, 300, 320, "f32"),
+                                      (300, 600, 2560, "bf16")])
+def test_host_entry_point(tw, M, N, K, dt):
+    """bitnet_w158a8_matmul_host (pinned host input and output, one call)
+    gives exactly the device entry point's output, on the fused, mma.sync and
+    tensor-core paths, and the oracle's."""
+    rng = np.random.default_rng(M + N + K)
+    W = synth.latent_weights(rng, N, K)
+    x = rng.standard_t(3, (M, K)).astype(np.float32)
+    Xd, xexact = as_x(x, dt)
+    pd, gd, po, go = quantize_weights_both(W)
+    ydt = torch.float32 if dt == "f32" else torch.bfloat16
+    want_d = tw.bitnet_w158a8_matmul(Xd, pd, gd, out_dtype=ydt)
+    Xh = Xd.cpu().pin_memory()
+    Yh = torch.empty((M, N), dtype=ydt).pin_memory()
+    X2 = torch.empty_like(Xd)
+    Y2 = torch.empty((M, N), dtype=ydt, device=DEV)
+    for _ in range(2):
+        Yh.zero_()
+        tw.bitnet_w158a8_matmul_host(Xh, pd, gd, X2, Y2, Yh, weights_static=True)
+        assert torch.equal(Yh, want_d.cpu())
+    want_o = ref.bitlinear(xexact, po, go, N)["y"]
+    if dt == "f32":
+        assert np.array_equal(Yh.numpy(), want_o)
+    else:
+        assert np.array_equal(Yh.view(torch.int16).numpy().view(np.uint16), ref.to_bf16(want_o))
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
 def test_repeatable(tw):
     d = synth.config_inputs("sweep", M=8, proj=0)
     pd, gd = tw.bitnet_quantize_weights(f32_t(d["W"]))
