@@ -190,13 +190,13 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + 64);          // [kMaxSlots]
   float *red_a = reinterpret_cast<float *>(smem + 128);               // [kCWarps]
   double *red_s = reinterpret_cast<double *>(smem + 192);             // [kCWarps]
-  float *red_max = reinterpret_cast<float *>(smem + 384);             // [kCWarps]
   volatile int *stop = reinterpret_cast<volatile int *>(smem + 320);
   int *issued_sh = reinterpret_cast<int *>(smem + 324);
   int *consumed_sh = reinterpret_cast<int *>(smem + 328);
   // `stop` as thread 0 saw it before the last consumer barrier: the value
   // every consumer acts on, so that all of them leave the loop together.
   int *stop_snap = reinterpret_cast<int *>(smem + 332);
+  float *red_max = reinterpret_cast<float *>(smem + 384);             // [kCWarps]
   StepP *tab = reinterpret_cast<StepP *>(smem + kHeader);            // [n_steps]
   float *gam = reinterpret_cast<float *>(smem + kHeader + align128(P.n_steps * 48));
   int2 *rr = reinterpret_cast<int2 *>(smem + kHeader + align128(P.n_steps * 48) +
@@ -401,9 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       if (lane == 0) red_max[warp] = wmax;
       if (tid == 0) *stop_snap = *stop;
       consumers_sync();
-      // ---- warp 0 stores the CTA's outputs (two per 32-bit word), folds
-      // their max |y| (over what the next step reads) into the step's max
-      // word and counts the CTA in
+      // ---- every warp has stored its rows; warp 0 folds the CTA's max |y|
+      // (over what the next step reads) into the step's max word and counts
+      // the CTA in
       if (warp == 0 && !*stop_snap) {
         float la = lane < kCWarps ? red_max[lane] : 0.0f;
         la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
