@@ -12,20 +12,23 @@
 //     slots (one bulk copy per projection, L2 evict-first) as far ahead as the
 //     ring allows, while the consumer warps are still on earlier links.
 //   * A link's outputs go straight to that step's output buffer, each warp
-//     storing its finished rows at once.  Each CTA then folds the largest |y|
-//     among them (over the part the next step reads) into one 64-bit word
-//     per step with an atomic max (the launch's tag in the high half, the
-//     float's bits in the low half: non-negative floats order as their bit
-//     patterns, so the maximum is exact and independent of the order of the
-//     CTAs), and adds one to the step's arrival counter with release
-//     semantics (no separate fence: a fence also waits for the producer's
-//     bulk copies in flight).
-//   * Before step s + 1, one thread per CTA polls that counter (one word on
-//     its own line) until every CTA has arrived; then every thread loads its
-//     part of the input vector and the max word, in one round trip.  Where a
-//     layer starts (the weightless RMS normalisation), every CTA also sums
-//     the squares of the loaded input in fp64, all in the same fixed order,
-//     so all CTAs normalise identically.
+//     storing its finished rows at once.  The values the next step reads are
+//     also stored as tagged 32-bit words in the workspace: the bf16 value in
+//     the low half, a 16-bit tag of this launch in the high half, one
+//     single-copy-atomic store per value.  A word is valid once its tag is
+//     this launch's, so no fence has to order the data before the signal.
+//   * A warp that has stored its rows counts itself in (shared memory); the
+//     CTA's last warp adds one to the step's arrival counter (a relaxed add:
+//     no fence, which would also wait for the producer's bulk copies in
+//     flight), hands the weight slot back and polls the counter until every
+//     CTA has arrived.  One thread per CTA polls, so the L2 sees one load per
+//     CTA per round; the other warps wait at a CTA barrier.
+//   * Step s + 1 then loads its part of the tagged input (relaxed loads
+//     through L2); a word whose tag is not yet this launch's (the counter
+//     may be seen before the data) is loaded again, bounded.  Each CTA
+//     reduces the max |x| of the whole input itself, and where a layer
+//     starts (the weightless RMS normalisation) the fp64 sum of squares, all
+//     in the same fixed order in every CTA, so all CTAs quantise identically.
 //   * Per link, each CTA quantises the whole input to int8 exactly as
 //     bitnet_quantize_act does and computes its balanced range of output
 //     features with the byte-permute unpack and dp4a, in the same int32
@@ -33,10 +36,14 @@
 //     w takes rows w, w + 16, ... of the CTA's range, up to 4 at a time: a
 //     lane loads each of its activation chunks once per pass and uses it for
 //     all of the pass's rows, and stores each row as soon as it is done.
-//   * The counters only grow: launch T (T = the launch counter kept in the
-//     workspace, plus one) waits for T * ctas arrivals; CTA 0 advances the
-//     launch counter once all CTAs have passed the last step, so graph
-//     replays and repeated calls need no host action.
+//   * Launch T (T = the launch counter kept in the workspace, plus one) tags
+//     its words with (T mod 65535) + 1, never 0 (a zero-filled workspace
+//     holds no valid word) and different from the previous launch's tag, and
+//     waits for T * ctas arrivals (the counters only grow).  The last step
+//     is counted with release semantics after a CTA barrier; CTA 0 waits for
+//     it with acquire loads, normalises the last output (optional) and
+//     advances the launch counter, so graph replays and repeated calls need
+//     no host action.
 // Every wait is bounded: a poll, an mbarrier wait or the final counter wait
 // that gives up records BITNET_ERR_TIMEOUT and the CTA stops at the next
 // step boundary, after its bulk copies in flight have landed.
@@ -71,7 +78,7 @@ struct __align__(8) StepP {
   uint16_t *Xn;      // bf16 [K] normalised input, or null
   int N, K;
   int flags;         // kStepRelu2 | kStepNormIn
-  int pad;
+  int toff;          // first tagged word of this step's output (the part the next step reads)
 };
 
 struct ChainP {
@@ -79,21 +86,29 @@ struct ChainP {
   uint16_t *y_norm;
   unsigned *epoch;
   unsigned *arrive;           // [n_steps], one per 128-byte line
-  unsigned long long *amax;   // [n_steps], one per 128-byte line: tag << 32 | max |y| bits
+  uint32_t *tagged;           // tag << 16 | bf16 bits, per step from toff
   int *status;
   int n_steps, ctas, slots, slot_bytes, xq_bytes, y_norm_n;
   StepP steps[kChainMaxSteps];
 };
 
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
 __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
   unsigned v;
   asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+// Four tagged words written by other SMs in this launch (each word is read
+// single-copy atomic, the four need not be from the same moment).
+__device__ __forceinline__ uint4 ld_relaxed_u4(const uint32_t *p) {
+  uint4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u32(uint32_t *p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 // 16 bytes from global memory through L2 only (another SM wrote them in this
 // launch; nothing of them may come from this SM's L1).
@@ -104,6 +119,9 @@ __device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
                : "l"(p)
                : "memory");
   return v;
+}
+__device__ __forceinline__ void red_relaxed_add(unsigned *p, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -127,8 +145,8 @@ __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32
       : "memory");
 }
 
-// Rows [r0, r1) of an N-row projection owned by CTA c: whole pairs of rows
-// (one 32-bit store each), balanced over the CTAs.
+// Rows [r0, r1) of an N-row projection owned by CTA c: whole pairs of rows,
+// balanced over the CTAs.
 __host__ __device__ inline void cta_rows(int N, int c, int ctas, int &r0, int &r1) {
   const long long pairs = (N + 1) / 2;
   r0 = static_cast<int>(2 * (pairs * c / ctas));
@@ -136,7 +154,6 @@ __host__ __device__ inline void cta_rows(int N, int c, int ctas, int &r0, int &r
   r1 = e < N ? e : N;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ uint32_t bf16_bits(float y) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(y)));
 }
@@ -151,18 +168,24 @@ __device__ __forceinline__ void chunk_to_float(uint4 u, float (&v)[8]) {
     v[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
   }
 }
+// True when all four words carry the tag `tb` (already shifted to the high half).
+__device__ __forceinline__ bool tagged_ok(uint4 u, uint32_t tb) {
+  return (((u.x ^ tb) | (u.y ^ tb) | (u.z ^ tb) | (u.w ^ tb)) >> 16) == 0u;
+}
 
-// Bounded wait (one thread) until the step's arrival counter reaches
-// `target`, polling with acquire loads: what every CTA stored before
-// arriving is then visible to this thread (and, after a CTA barrier, to the
-// whole CTA).  Acquire loads instead of relaxed ones and a fence: the fence
-// also waits for this SM's memory operations in flight, among them the
-// producer's bulk copies (measured: 627 -> 580 us per token).
-__device__ __forceinline__ bool wait_arrivals(const unsigned *ctr, unsigned target, int *status) {
+// Bounded wait (one thread) until a counter reaches `target`.  ACQUIRE:
+// with acquire loads, so that what every CTA stored before its release add
+// is then visible to this thread (and, after a CTA barrier, to the whole
+// CTA); else relaxed loads (the data it announces carries its own tags).
+template <bool ACQUIRE>
+__device__ __forceinline__ bool wait_count(const unsigned *ctr, unsigned target, int *status) {
   const long long t0 = clock64();
   while (true) {
     unsigned v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (ACQUIRE)
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    else
+      asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v == target) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       record_status(status, kStatusTimeout);
@@ -186,19 +209,84 @@ __device__ __forceinline__ bool wait_or_stop(uint64_t *bar, uint32_t parity,
   }
 }
 
+// This thread's part of a step's input from the tagged words `src` (8 values
+// per chunk, chunks tid, tid + 512, ...): load every word once, then re-load
+// the 4-word groups whose tag is not yet `tb` until all of them carry it.
+// Bounded: false (and BITNET_ERR_TIMEOUT recorded) if they never do.
+__device__ __forceinline__ bool load_tagged(const uint32_t *src, int nchunks, int tid, uint32_t tb,
+                                            float (&v)[kChunks][8], int *status) {
+  uint4 t[kChunks][2];
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    const int c = tid + i * kCThreads;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      t[i][h] = c < nchunks ? ld_relaxed_u4(src + 8 * c + 4 * h) : make_uint4(tb, tb, tb, tb);
+  }
+  const long long t0 = clock64();
+  bool ok = true;
+  while (true) {
+    bool all = true;
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) all = all && tagged_ok(t[i][h], tb);
+    if (all) break;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      record_status(status, kStatusTimeout);
+      ok = false;
+      break;
+    }
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+      const int c = tid + i * kCThreads;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (!tagged_ok(t[i][h], tb)) t[i][h] = ld_relaxed_u4(src + 8 * c + 4 * h);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t w[4] = {t[i][h].x, t[i][h].y, t[i][h].z, t[i][h].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[i][4 * h + e] = __uint_as_float(w[e] << 16);
+    }
+  return ok;
+}
+
+// NR rows of a pass (rows w, w + 16, ... from `wr`, each `words` packed
+// words long) against the quantised input: lane l takes words l, l + 32, ...
+template <int NR>
+__device__ __forceinline__ void dot_rows(const uint32_t *wr, int words, const uint4 *xq4, int lane,
+                                         int (&acc)[kRowsPerPass]) {
+  const size_t stride = static_cast<size_t>(kCWarps) * words;
+  for (int w = lane; w < words; w += 32) {
+    const uint4 x = xq4[w];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) acc[i] = dot_word(unpack_word(wr[i * stride + w]), x, acc[i]);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constant__ ChainP P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);                // [kMaxSlots]
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + 64);          // [kMaxSlots]
   float *red_a = reinterpret_cast<float *>(smem + 128);               // [kCWarps]
   double *red_s = reinterpret_cast<double *>(smem + 192);             // [kCWarps]
+  // set by the producer when it gives up, and by consumers when they halt
   volatile int *stop = reinterpret_cast<volatile int *>(smem + 320);
   int *issued_sh = reinterpret_cast<int *>(smem + 324);
   int *consumed_sh = reinterpret_cast<int *>(smem + 328);
-  // `stop` as thread 0 saw it before the last consumer barrier: the value
-  // every consumer acts on, so that all of them leave the loop together.
-  int *stop_snap = reinterpret_cast<int *>(smem + 332);
-  float *red_max = reinterpret_cast<float *>(smem + 384);             // [kCWarps]
+  // set by consumer threads only, before a consumer barrier, and read by all
+  // of them after it: every consumer leaves the loop at the same step
+  volatile int *halt = reinterpret_cast<volatile int *>(smem + 332);
+  volatile int *fin = reinterpret_cast<volatile int *>(smem + 336);  // CTA 0: every CTA done
+  int *counted = reinterpret_cast<int *>(smem + 340);                // warps done with the step
+  // `halt` as the step's last warp saw it before the CTA barrier that ends
+  // the step (read by all after that barrier)
+  volatile int *halt_snap = reinterpret_cast<volatile int *>(smem + 344);
   StepP *tab = reinterpret_cast<StepP *>(smem + kHeader);            // [n_steps]
   float *gam = reinterpret_cast<float *>(smem + kHeader + align128(P.n_steps * 48));
   int2 *rr = reinterpret_cast<int2 *>(smem + kHeader + align128(P.n_steps * 48) +
@@ -214,7 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       mbar_init(empty + i, 1);
     }
     *stop = 0;
-    *stop_snap = 0;
+    *halt = 0;
+    *halt_snap = 0;
+    *counted = 0;
     *issued_sh = 0;
     *consumed_sh = 0;
     fence_barrier_init();
@@ -265,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   } else {
     // ---------------------------------------------------------- consumers
     const unsigned tag = ld_relaxed_u32(P.epoch) + 1u;
+    const uint32_t tb = (tag % 0xFFFFu + 1u) << 16;
     const unsigned target = tag * static_cast<unsigned>(P.ctas);
     int consumed = 0, slot = 0;
     uint32_t phase = 0;  // parity of the slot's fill to wait for
@@ -272,66 +363,45 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       const StepP &d = tab[s];
       const int nchunks = d.K >> 3;  // 8 bf16 values per chunk
       const bool norm = (d.flags & kStepNormIn) != 0;
-      // ---- the input: x0, or the previous step's output once every CTA has stored it
-      const uint16_t *src = s == 0 ? P.x0 : tab[s - 1].Y;
-      if (s > 0) {
-        if (tid == 0 && !*stop &&
-            !wait_arrivals(P.arrive + static_cast<size_t>(s - 1) * 32, target, P.status))
-          *stop = 1;
-        if (tid == 0) *stop_snap = *stop;
-        consumers_sync();
-        if (*stop_snap) break;
-      }
-      uint4 raw[kChunks];
-#pragma unroll
-      for (int i = 0; i < kChunks; ++i) {
-        const int c = tid + i * kCThreads;
-        raw[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (c < nchunks)
-          raw[i] = s == 0 ? *reinterpret_cast<const uint4 *>(src + 8 * c) : ld_cg_u4(src + 8 * c);
-      }
-      float a;
-      if (s > 0) {
-        // the exact max |x| the producers folded together (tag checked)
-        const unsigned long long m = ld_relaxed_u64(P.amax + static_cast<size_t>(s - 1) * 16);
-        a = static_cast<unsigned>(m >> 32) == tag ? __uint_as_float(static_cast<uint32_t>(m)) : 0.0f;
-      } else {
-        float la = 0.0f;
+      // ---- the input: x0, or the previous step's tagged output
+      float v[kChunks][8];
+      if (s == 0) {
 #pragma unroll
         for (int i = 0; i < kChunks; ++i) {
-          float v[8];
-          chunk_to_float(raw[i], v);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) la = fmaxf(la, fabsf(v[e]));
+          const int c = tid + i * kCThreads;
+          chunk_to_float(c < nchunks ? *reinterpret_cast<const uint4 *>(P.x0 + 8 * c)
+                                     : make_uint4(0u, 0u, 0u, 0u),
+                         v[i]);
         }
-        la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
-        if (lane == 0) red_a[warp] = la;
+      } else {
+        if (*halt_snap) break;
+        if (!load_tagged(P.tagged + tab[s - 1].toff, nchunks, tid, tb, v, P.status)) *halt = 1;
       }
+      float la = 0.0f;
+      double ss = 0.0;
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          la = fmaxf(la, fabsf(v[i][e]));
+          if (norm) ss = add_sq(ss, v[i][e]);  // fp64, the same order in every CTA
+        }
+      la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
+      if (norm) ss = warp_sum_f64(ss);
+      if (lane == 0) {
+        red_a[warp] = la;
+        red_s[warp] = ss;
+      }
+      consumers_sync();
+      if (*halt) break;
+      float a = __uint_as_float(
+          __reduce_max_sync(0xffffffffu, __float_as_uint(lane < kCWarps ? red_a[lane] : 0.0f)));
       float inv = 1.0f;
       if (norm) {
-        // sum of squares of the whole input, fp64, the same order in every CTA
-        double ss = 0.0;
-#pragma unroll
-        for (int i = 0; i < kChunks; ++i) {
-          float v[8];
-          chunk_to_float(raw[i], v);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ss = add_sq(ss, v[e]);
-        }
-        ss = warp_sum_f64(ss);
-        if (lane == 0) red_s[warp] = ss;
-      }
-      if (s == 0 || norm) {
-        consumers_sync();
-        if (s == 0)
-          a = __uint_as_float(__reduce_max_sync(
-              0xffffffffu, __float_as_uint(lane < kCWarps ? red_a[lane] : 0.0f)));
-        if (norm) {
-          inv = rms_factor(warp_sum_f64(lane < kCWarps ? red_s[lane] : 0.0), d.K);
-          // rounding x * inv to bf16 is monotone in |x|: the max of the
-          // normalised values is the normalised max
-          a = round_bf16(__fmul_rn(a, inv));
-        }
+        inv = rms_factor(warp_sum_f64(lane < kCWarps ? red_s[lane] : 0.0), d.K);
+        // rounding x * inv to bf16 is monotone in |x|: the max of the
+        // normalised values is the normalised max
+        a = round_bf16(__fmul_rn(a, inv));
       }
       const float sc = act_scale(a);
       const float r = __fdiv_rn(gam[s], sc);
@@ -341,20 +411,18 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         const int c0 = i * kCThreads;
         if (c0 >= nchunks) break;  // uniform over the CTA
         const int c = c0 + tid;
-        float v[8];
-        chunk_to_float(raw[i], v);
         if (norm) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = round_bf16(__fmul_rn(v[e], inv));
+          for (int e = 0; e < 8; ++e) v[i][e] = round_bf16(__fmul_rn(v[i][e], inv));
           if (d.Xn != nullptr && blockIdx.x == 0 && c < nchunks) {
             uint32_t o[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-              o[h] = (__float_as_uint(v[2 * h]) >> 16) | (__float_as_uint(v[2 * h + 1]) & 0xFFFF0000u);
+              o[h] = (__float_as_uint(v[i][2 * h]) >> 16) | (__float_as_uint(v[i][2 * h + 1]) & 0xFFFF0000u);
             *reinterpret_cast<uint4 *>(d.Xn + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
-        store_half_group(xq, c, v, sc, c < nchunks);
+        store_half_group(xq, c, v[i], sc, c < nchunks);
       }
       consumers_sync();
       // ---- this CTA's rows: warp w takes rows w, w + 16, ... of its range
@@ -364,89 +432,82 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       const int words = d.K >> 4;  // packed 32-bit words per row
       const bool last = s + 1 == P.n_steps;
       const int k_next = last ? 0 : tab[s + 1].K;
+      uint32_t *tout = P.tagged + d.toff;
       const bool relu2 = (d.flags & kStepRelu2) != 0;
-      float wmax = 0.0f;  // this warp's max |y| over stored rows that the next step reads
       if (have_w) {
         consumed = s + 1;
         const uint32_t *wsl =
             reinterpret_cast<const uint32_t *>(slots + static_cast<size_t>(slot) * P.slot_bytes);
         for (int rb = warp; rb < rows; rb += kCWarps * kRowsPerPass) {
-          int acc[kRowsPerPass];
-#pragma unroll
-          for (int i = 0; i < kRowsPerPass; ++i) acc[i] = 0;
-          for (int w = lane; w < words; w += 32) {
-            const uint4 x = xq4[w];
-#pragma unroll
-            for (int i = 0; i < kRowsPerPass; ++i) {
-              const int rl = rb + i * kCWarps;
-              if (rl < rows) acc[i] = dot_word(unpack_word(wsl[static_cast<size_t>(rl) * words + w]), x, acc[i]);
-            }
-          }
+          int acc[kRowsPerPass] = {0, 0, 0, 0};
+          const uint32_t *wr = wsl + static_cast<size_t>(rb) * words;
+          const int nr = (rows - rb + kCWarps - 1) / kCWarps;  // rows in this pass (warp-uniform)
+          if (nr >= kRowsPerPass) dot_rows<kRowsPerPass>(wr, words, xq4, lane, acc);
+          else if (nr == 3) dot_rows<3>(wr, words, xq4, lane, acc);
+          else if (nr == 2) dot_rows<2>(wr, words, xq4, lane, acc);
+          else dot_rows<1>(wr, words, xq4, lane, acc);
 #pragma unroll
           for (int i = 0; i < kRowsPerPass; ++i) {
             const int rl = rb + i * kCWarps;
             if (rl < rows) {  // the same for the whole warp
               const int v = __reduce_add_sync(0xffffffffu, acc[i]);
-              if (lane == 0) {  // the row is complete: store it now
+              if (lane == i) {  // the row is complete: lane i stores it now
+                const int row = r0 + rl;
                 const uint32_t y = bf16_bits(epilogue_value(v, r, relu2));
-                d.Y[r0 + rl] = static_cast<uint16_t>(y);
-                if (r0 + rl < k_next) wmax = fmaxf(wmax, fabsf(bf16_lo(y)));
+                d.Y[row] = static_cast<uint16_t>(y);
+                if (row < k_next) st_relaxed_u32(tout + row, tb | y);
               }
             }
           }
         }
       } else {
-        *stop = 1;  // acted on at the next step's first barrier
+        *halt = 1;  // acted on when the step ends
       }
-      if (lane == 0) red_max[warp] = wmax;
-      if (tid == 0) *stop_snap = *stop;
-      consumers_sync();
-      // ---- every warp has stored its rows; warp 0 folds the CTA's max |y|
-      // (over what the next step reads) into the step's max word and counts
-      // the CTA in
-      if (warp == 0 && !*stop_snap) {
-        float la = lane < kCWarps ? red_max[lane] : 0.0f;
-        la = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(la)));
+      if (!last) {
+        // ---- count the warp in; the CTA's last warp hands the slot back,
+        // counts the CTA in and waits for every CTA (the others wait for it
+        // at the barrier below)
         __syncwarp();
+        int n_in = 0;
         if (lane == 0) {
-          if (!last && (r0 < k_next || blockIdx.x == 0))  // no value returned: nothing to wait for
-            asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(
-                             P.amax + static_cast<size_t>(s) * 16),
-                         "l"((static_cast<unsigned long long>(tag) << 32) | __float_as_uint(la))
-                         : "memory");
-          // release: every warp's stores (ordered before this thread by the
-          // barrier above) and the max are visible before the count; no
-          // separate fence, which would also wait for the bulk copies in
-          // flight (measured: 580 -> 561 us per token)
-          red_release_add(P.arrive + static_cast<size_t>(s) * 32, 1u);
+          asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                       : "=r"(n_in) : "r"(smem_u32(counted)) : "memory");
         }
+        n_in = __shfl_sync(0xffffffffu, n_in, 0);
+        if (n_in == kCWarps - 1 && lane == 0) {
+          *counted = 0;
+          const bool h = *halt != 0;
+          if (!h) {
+            mbar_arrive(empty + slot);  // every warp is past its reads of the slot
+            red_relaxed_add(P.arrive + static_cast<size_t>(s) * 32, 1u);
+            if (!wait_count<false>(P.arrive + static_cast<size_t>(s) * 32, target, P.status))
+              *halt = 1;
+          }
+          *halt_snap = *halt;
+        }
+        consumers_sync();
       }
-      // The slot is free once every warp is past the consumer barrier above;
-      // it is handed back only now, so that the producer's next bulk copy is
-      // not in flight while thread 0's fence waits for the step's stores
-      // (measured: 657 -> 627 us per token for the 30-layer chain).
-      if (tid == 0 && have_w) mbar_arrive(empty + slot);
       if (++slot == P.slots) {
         slot = 0;
         phase ^= 1u;
       }
     }
+    // ---- end of the chain: every CTA counts itself in for the last step
+    // once all its warps have stored their rows (release, after a CTA
+    // barrier); CTA 0 waits for all of them (acquire), normalises the last
+    // output (optional) and then advances the launch counter.
+    consumers_sync();
+    const bool halted = *halt != 0;
     if (tid == 0) {
       *consumed_sh = consumed;
-      *stop_snap = *stop;
+      if (halted) *stop = 1;  // the producer stops waiting for slots
+      else red_release_add(P.arrive + static_cast<size_t>(P.n_steps - 1) * 32, 1u);
     }
-
-    // ---- end of the chain: CTA 0 waits for every CTA's last outputs,
-    // normalises them (optional) and then advances the launch counter.
-    consumers_sync();
-    if (blockIdx.x == 0 && !*stop_snap) {
-      if (tid == 0) {
-        if (!wait_arrivals(P.arrive + static_cast<size_t>(P.n_steps - 1) * 32, target, P.status))
-          *stop = 1;
-        *stop_snap = *stop;
-      }
+    if (blockIdx.x == 0 && !halted) {
+      if (tid == 0)
+        *fin = wait_count<true>(P.arrive + static_cast<size_t>(P.n_steps - 1) * 32, target, P.status);
       consumers_sync();
-      if (!*stop_snap) {
+      if (*fin) {
         if (P.y_norm != nullptr) {
           const uint16_t *src = tab[P.n_steps - 1].Y;
           const int nchunks = P.y_norm_n >> 3;
@@ -456,10 +517,10 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
           for (int i = 0; i < kChunks; ++i) {
             const int c = tid + i * kCThreads;
             raw[i] = c < nchunks ? ld_cg_u4(src + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
-            float v[8];
-            chunk_to_float(raw[i], v);
+            float f[8];
+            chunk_to_float(raw[i], f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = add_sq(ss, v[e]);
+            for (int e = 0; e < 8; ++e) ss = add_sq(ss, f[e]);
           }
           ss = warp_sum_f64(ss);
           if (lane == 0) red_s[warp] = ss;
@@ -469,12 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
           for (int i = 0; i < kChunks; ++i) {
             const int c = tid + i * kCThreads;
             if (c >= nchunks) break;
-            float v[8];
-            chunk_to_float(raw[i], v);
+            float f[8];
+            chunk_to_float(raw[i], f);
             uint32_t o[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-              o[h] = bf16_bits(__fmul_rn(v[2 * h], iv)) | (bf16_bits(__fmul_rn(v[2 * h + 1], iv)) << 16);
+              o[h] = bf16_bits(__fmul_rn(f[2 * h], iv)) | (bf16_bits(__fmul_rn(f[2 * h + 1], iv)) << 16);
             *reinterpret_cast<uint4 *>(P.y_norm + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
@@ -532,8 +593,8 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   p.epoch = reinterpret_cast<unsigned *>(ws);
   p.arrive = reinterpret_cast<unsigned *>(ws + kChainWorkspaceHeader);
-  p.amax = reinterpret_cast<unsigned long long *>(ws + kChainWorkspaceHeader +
-                                                  static_cast<size_t>(n_steps) * kChainLine);
+  p.tagged = reinterpret_cast<uint32_t *>(ws + kChainWorkspaceHeader +
+                                          static_cast<size_t>(n_steps) * kChainLine);
   p.status = ctx.status;
   p.n_steps = n_steps;
   p.ctas = plan.ctas;
@@ -541,6 +602,7 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
   p.slot_bytes = plan.slot_bytes;
   p.xq_bytes = plan.xq_bytes;
   p.y_norm_n = static_cast<int>(y_norm_n);
+  int64_t toff = 0;
   for (int s = 0; s < n_steps; ++s) {
     StepP &d = p.steps[s];
     d.packed = steps[s].packed;
@@ -550,7 +612,8 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
     d.N = static_cast<int>(steps[s].N);
     d.K = static_cast<int>(steps[s].K);
     d.flags = static_cast<int>(steps[s].flags);
-    d.pad = 0;
+    d.toff = static_cast<int>(toff);
+    if (s + 1 < n_steps) toff += chain_tag_words(steps[s + 1].K);
   }
   cudaError_t e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(plan.smem));

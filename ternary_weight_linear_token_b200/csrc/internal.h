@@ -102,12 +102,14 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
 constexpr int kChainMaxSteps = 256;
 constexpr int kStepRelu2 = 1;
 constexpr int kStepNormIn = 2;
-constexpr size_t kChainWorkspaceHeader = 256;  // the launch counter at byte 0
 constexpr int kChainMaxCtas = 256;              // CTAs of one chain launch, at most
-// After the header, one 128-byte line per step holding its arrival counter,
-// then one per step holding its tagged max |y| word.
+// Workspace: the launch counter at byte 0; after the 256-byte header one
+// 128-byte line per step holding its arrival counter; then for every step
+// but the last the tagged words of the part of its output the next step
+// reads (its K values), each step's run a whole number of 128-byte lines.
+constexpr size_t kChainWorkspaceHeader = 256;
 constexpr size_t kChainLine = 128;
-inline size_t chain_sync_bytes(int n_steps) { return 2 * kChainLine * static_cast<size_t>(n_steps); }
+inline int64_t chain_tag_words(int64_t k_next) { return (k_next + 31) / 32 * 32; }
 struct ChainStep {
   const uint8_t *packed;
   const float *gamma;
