@@ -348,14 +348,13 @@ bitnet_status bitnet_rms_norm(const void *X, bitnet_dtype x_dtype, int64_t M, in
  *   y_norm     bf16 [steps[n-1].N] or NULL: the RMS normalisation of the
  *              last step's output (N % 16 == 0 and N <= 8192 when given).
  *   workspace  >= bitnet_decode_chain_workspace_size(steps, n_steps) bytes
- *              (256 + 128 * n_steps + 4 * the sum of K over steps
- *              1 .. n_steps-1, rounded up to 256), 16-byte aligned.
- *              ZERO-FILLED before the first call; then passed unchanged to
- *              every later call of a chain (the library keeps a launch
- *              counter and per-step arrival counters in it, which only grow,
- *              and every link's values tagged with the launch they belong
- *              to).  After a call that reported BITNET_ERR_TIMEOUT, zero it
- *              again.
+ *              (256 + 4 * the sum of K over steps 1 .. n_steps-1, rounded
+ *              up to 256), 16-byte aligned.  ZERO-FILLED before the first
+ *              call; then passed unchanged to every later call of a chain
+ *              (the library keeps a launch counter and a done counter in it,
+ *              which only grow, and every link's values tagged with the
+ *              launch they belong to).  After a call that reported
+ *              BITNET_ERR_TIMEOUT, zero it again.
  *              Two chains must not run concurrently on one workspace.
  * Per step: packed [N][K/4] and gamma as from bitnet_quantize_weights
  * (packed 16-byte aligned); Y bf16 [N], 16-byte aligned; 1 <= N <= 2^22;

@@ -266,8 +266,7 @@ bitnet_status check_chain(const bitnet_chain_step *steps, int n_steps) {
 size_t chain_workspace(const bitnet_chain_step *steps, int n_steps) {
   int64_t words = 0;
   for (int s = 1; s < n_steps; ++s) words += chain_tag_words(steps[s].K);
-  return align256(kChainWorkspaceHeader + kChainLine * static_cast<size_t>(n_steps) +
-                  4 * static_cast<size_t>(words));
+  return align256(kChainWorkspaceHeader + 4 * static_cast<size_t>(words));
 }
 
 }  // namespace

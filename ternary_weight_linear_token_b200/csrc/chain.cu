@@ -16,19 +16,16 @@
 //     also stored as tagged 32-bit words in the workspace: the bf16 value in
 //     the low half, a 16-bit tag of this launch in the high half, one
 //     single-copy-atomic store per value.  A word is valid once its tag is
-//     this launch's, so no fence has to order the data before the signal.
-//   * A warp that has stored its rows counts itself in (shared memory); the
-//     CTA's last warp adds one to the step's arrival counter (a relaxed add:
-//     no fence, which would also wait for the producer's bulk copies in
-//     flight), hands the weight slot back and polls the counter until every
-//     CTA has arrived.  One thread per CTA polls, so the L2 sees one load per
-//     CTA per round; the other warps wait at a CTA barrier.
-//   * Step s + 1 then loads its part of the tagged input (relaxed loads
-//     through L2); a word whose tag is not yet this launch's (the counter
-//     may be seen before the data) is loaded again, bounded.  Each CTA
-//     reduces the max |x| of the whole input itself, and where a layer
-//     starts (the weightless RMS normalisation) the fp64 sum of squares, all
-//     in the same fixed order in every CTA, so all CTAs quantise identically.
+//     this launch's, so the data carries its own readiness: no arrival
+//     counter, no fence, no flag to order the data before.
+//   * When all its warps have stored their rows (a CTA barrier, so that no
+//     warp polls while others of the SM still compute), the CTA hands the
+//     weight slot back and starts the next step: every thread loads its part
+//     of the tagged input (relaxed loads through L2) and loads again the
+//     words whose tag is not yet this launch's, bounded.  Each CTA reduces
+//     the max |x| of the whole input itself, and where a layer starts (the
+//     weightless RMS normalisation) the fp64 sum of squares, all in the same
+//     fixed order in every CTA, so all CTAs quantise identically.
 //   * Per link, each CTA quantises the whole input to int8 exactly as
 //     bitnet_quantize_act does and computes its balanced range of output
 //     features with the byte-permute unpack and dp4a, in the same int32
@@ -38,12 +35,12 @@
 //     all of the pass's rows, and stores each row as soon as it is done.
 //   * Launch T (T = the launch counter kept in the workspace, plus one) tags
 //     its words with (T mod 65535) + 1, never 0 (a zero-filled workspace
-//     holds no valid word) and different from the previous launch's tag, and
-//     waits for T * ctas arrivals (the counters only grow).  The last step
-//     is counted with release semantics after a CTA barrier; CTA 0 waits for
-//     it with acquire loads, normalises the last output (optional) and
-//     advances the launch counter, so graph replays and repeated calls need
-//     no host action.
+//     holds no valid word) and different from the previous launch's tag.
+//     After the last step every CTA adds one to a done counter that only
+//     grows (release, after a CTA barrier); CTA 0 waits for T * ctas
+//     (acquire), normalises the last output (optional) and advances the
+//     launch counter, so graph replays and repeated calls need no host
+//     action.
 // Every wait is bounded: a poll, an mbarrier wait or the final counter wait
 // that gives up records BITNET_ERR_TIMEOUT and the CTA stops at the next
 // step boundary, after its bulk copies in flight have landed.
@@ -63,6 +60,7 @@ constexpr int kHeader = 1024;
 constexpr int kBarConsumers = 1;            // named barrier of the consumer warps
 constexpr int kChunks = 2;                  // 8-element input chunks per thread: K <= 8192
 constexpr int kRowsPerPass = 4;             // rows a warp carries at once in the dot products
+constexpr unsigned kFirstPollDelayNs = 300;  // before a step's first input loads
 
 __host__ __device__ constexpr int align128(int n) { return (n + 127) / 128 * 128; }
 // Shared-memory copies made once at the start: the step descriptors, every
@@ -85,7 +83,7 @@ struct ChainP {
   const uint16_t *x0;
   uint16_t *y_norm;
   unsigned *epoch;
-  unsigned *arrive;           // [n_steps], one per 128-byte line
+  unsigned *done;             // CTAs past the last step, summed over launches
   uint32_t *tagged;           // tag << 16 | bf16 bits, per step from toff
   int *status;
   int n_steps, ctas, slots, slot_bytes, xq_bytes, y_norm_n;
@@ -119,9 +117,6 @@ __device__ __forceinline__ uint4 ld_cg_u4(const void *p) {
                : "l"(p)
                : "memory");
   return v;
-}
-__device__ __forceinline__ void red_relaxed_add(unsigned *p, unsigned v) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -173,19 +168,14 @@ __device__ __forceinline__ bool tagged_ok(uint4 u, uint32_t tb) {
   return (((u.x ^ tb) | (u.y ^ tb) | (u.z ^ tb) | (u.w ^ tb)) >> 16) == 0u;
 }
 
-// Bounded wait (one thread) until a counter reaches `target`.  ACQUIRE:
-// with acquire loads, so that what every CTA stored before its release add
-// is then visible to this thread (and, after a CTA barrier, to the whole
-// CTA); else relaxed loads (the data it announces carries its own tags).
-template <bool ACQUIRE>
+// Bounded wait (one thread) until a counter reaches `target`, polling with
+// acquire loads: what every CTA stored before its release add is then
+// visible to this thread (and, after a CTA barrier, to the whole CTA).
 __device__ __forceinline__ bool wait_count(const unsigned *ctr, unsigned target, int *status) {
   const long long t0 = clock64();
   while (true) {
     unsigned v;
-    if (ACQUIRE)
-      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-    else
-      asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v == target) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       record_status(status, kStatusTimeout);
@@ -216,6 +206,12 @@ __device__ __forceinline__ bool wait_or_stop(uint64_t *bar, uint32_t parity,
 __device__ __forceinline__ bool load_tagged(const uint32_t *src, int nchunks, int tid, uint32_t tb,
                                             float (&v)[kChunks][8], int *status) {
   uint4 t[kChunks][2];
+  // The first loads wait about 0.3 us: polling the moment the CTA is done,
+  // while the last CTAs still store, slowed every step (30-layer stack: 575
+  // us per token without the delay, 548 / 480 / 447 / 462 / 458 with 50 /
+  // 150 / 300 / 600 / 1000 ns; sleeping only after a first poll that found
+  // missing words: 705).
+  __nanosleep(kFirstPollDelayNs);
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
     const int c = tid + i * kCThreads;
@@ -258,15 +254,28 @@ __device__ __forceinline__ bool load_tagged(const uint32_t *src, int nchunks, in
 
 // NR rows of a pass (rows w, w + 16, ... from `wr`, each `words` packed
 // words long) against the quantised input: lane l takes words l, l + 32, ...
+// Two accumulators per row halve the chain of dependent dp4a (integer sums:
+// the order does not change the result; 444 -> 436 us per token).
 template <int NR>
 __device__ __forceinline__ void dot_rows(const uint32_t *wr, int words, const uint4 *xq4, int lane,
                                          int (&acc)[kRowsPerPass]) {
   const size_t stride = static_cast<size_t>(kCWarps) * words;
+  int acc2[NR];
+#pragma unroll
+  for (int i = 0; i < NR; ++i) acc2[i] = 0;
   for (int w = lane; w < words; w += 32) {
     const uint4 x = xq4[w];
 #pragma unroll
-    for (int i = 0; i < NR; ++i) acc[i] = dot_word(unpack_word(wr[i * stride + w]), x, acc[i]);
+    for (int i = 0; i < NR; ++i) {
+      const Unpacked q = unpack_word(wr[i * stride + w]);
+      acc[i] = __dp4a(q.a, static_cast<int>(x.x), acc[i]);
+      acc2[i] = __dp4a(q.b, static_cast<int>(x.y), acc2[i]);
+      acc[i] = __dp4a(q.c, static_cast<int>(x.z), acc[i]);
+      acc2[i] = __dp4a(q.d, static_cast<int>(x.w), acc2[i]);
+    }
   }
+#pragma unroll
+  for (int i = 0; i < NR; ++i) acc[i] += acc2[i];
 }
 
 __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constant__ ChainP P) {
@@ -279,14 +288,14 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
   volatile int *stop = reinterpret_cast<volatile int *>(smem + 320);
   int *issued_sh = reinterpret_cast<int *>(smem + 324);
   int *consumed_sh = reinterpret_cast<int *>(smem + 328);
-  // set by consumer threads only, before a consumer barrier, and read by all
-  // of them after it: every consumer leaves the loop at the same step
-  volatile int *halt = reinterpret_cast<volatile int *>(smem + 332);
-  volatile int *fin = reinterpret_cast<volatile int *>(smem + 336);  // CTA 0: every CTA done
-  int *counted = reinterpret_cast<int *>(smem + 340);                // warps done with the step
-  // `halt` as the step's last warp saw it before the CTA barrier that ends
-  // the step (read by all after that barrier)
-  volatile int *halt_snap = reinterpret_cast<volatile int *>(smem + 344);
+  // Set by consumer threads only, each before the consumer barrier after
+  // which all of them read it, and not again before all have: every
+  // consumer leaves the loop at the same step.  halt_in: an input poll gave
+  // up (read after the reduction barrier); halt_w: a weight slot never
+  // landed (read after the step's last barrier).
+  volatile int *halt_in = reinterpret_cast<volatile int *>(smem + 332);
+  volatile int *halt_w = reinterpret_cast<volatile int *>(smem + 336);
+  volatile int *fin = reinterpret_cast<volatile int *>(smem + 340);  // CTA 0: every CTA done
   StepP *tab = reinterpret_cast<StepP *>(smem + kHeader);            // [n_steps]
   float *gam = reinterpret_cast<float *>(smem + kHeader + align128(P.n_steps * 48));
   int2 *rr = reinterpret_cast<int2 *>(smem + kHeader + align128(P.n_steps * 48) +
@@ -302,9 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
       mbar_init(empty + i, 1);
     }
     *stop = 0;
-    *halt = 0;
-    *halt_snap = 0;
-    *counted = 0;
+    *halt_in = 0;
+    *halt_w = 0;
     *issued_sh = 0;
     *consumed_sh = 0;
     fence_barrier_init();
@@ -356,7 +364,6 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
     // ---------------------------------------------------------- consumers
     const unsigned tag = ld_relaxed_u32(P.epoch) + 1u;
     const uint32_t tb = (tag % 0xFFFFu + 1u) << 16;
-    const unsigned target = tag * static_cast<unsigned>(P.ctas);
     int consumed = 0, slot = 0;
     uint32_t phase = 0;  // parity of the slot's fill to wait for
     for (int s = 0; s < P.n_steps; ++s) {
@@ -374,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
                          v[i]);
         }
       } else {
-        if (*halt_snap) break;
-        if (!load_tagged(P.tagged + tab[s - 1].toff, nchunks, tid, tb, v, P.status)) *halt = 1;
+        if (*halt_w) break;
+        if (!load_tagged(P.tagged + tab[s - 1].toff, nchunks, tid, tb, v, P.status)) *halt_in = 1;
       }
       float la = 0.0f;
       double ss = 0.0;
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
         red_s[warp] = ss;
       }
       consumers_sync();
-      if (*halt) break;
+      if (*halt_in) break;
       float a = __uint_as_float(
           __reduce_max_sync(0xffffffffu, __float_as_uint(lane < kCWarps ? red_a[lane] : 0.0f)));
       float inv = 1.0f;
@@ -461,31 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
           }
         }
       } else {
-        *halt = 1;  // acted on when the step ends
+        *halt_w = 1;  // acted on when the step ends
       }
       if (!last) {
-        // ---- count the warp in; the CTA's last warp hands the slot back,
-        // counts the CTA in and waits for every CTA (the others wait for it
-        // at the barrier below)
-        __syncwarp();
-        int n_in = 0;
-        if (lane == 0) {
-          asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
-                       : "=r"(n_in) : "r"(smem_u32(counted)) : "memory");
-        }
-        n_in = __shfl_sync(0xffffffffu, n_in, 0);
-        if (n_in == kCWarps - 1 && lane == 0) {
-          *counted = 0;
-          const bool h = *halt != 0;
-          if (!h) {
-            mbar_arrive(empty + slot);  // every warp is past its reads of the slot
-            red_relaxed_add(P.arrive + static_cast<size_t>(s) * 32, 1u);
-            if (!wait_count<false>(P.arrive + static_cast<size_t>(s) * 32, target, P.status))
-              *halt = 1;
-          }
-          *halt_snap = *halt;
-        }
+        // every warp is past its reads of the slot and has stored its rows;
+        // no warp polls the next input while others still compute
         consumers_sync();
+        if (tid == 0 && !*halt_w) mbar_arrive(empty + slot);
       }
       if (++slot == P.slots) {
         slot = 0;
@@ -497,15 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1) chain_kernel(const __grid_constan
     // barrier); CTA 0 waits for all of them (acquire), normalises the last
     // output (optional) and then advances the launch counter.
     consumers_sync();
-    const bool halted = *halt != 0;
+    const bool halted = *halt_in != 0 || *halt_w != 0;
     if (tid == 0) {
       *consumed_sh = consumed;
       if (halted) *stop = 1;  // the producer stops waiting for slots
-      else red_release_add(P.arrive + static_cast<size_t>(P.n_steps - 1) * 32, 1u);
+      else red_release_add(P.done, 1u);
     }
     if (blockIdx.x == 0 && !halted) {
-      if (tid == 0)
-        *fin = wait_count<true>(P.arrive + static_cast<size_t>(P.n_steps - 1) * 32, target, P.status);
+      if (tid == 0) *fin = wait_count(P.done, tag * static_cast<unsigned>(P.ctas), P.status);
       consumers_sync();
       if (*fin) {
         if (P.y_norm != nullptr) {
@@ -592,9 +580,8 @@ cudaError_t launch_chain(const ChainStep *steps, int n_steps, const ChainPlan &p
   p.y_norm = static_cast<uint16_t *>(y_norm);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   p.epoch = reinterpret_cast<unsigned *>(ws);
-  p.arrive = reinterpret_cast<unsigned *>(ws + kChainWorkspaceHeader);
-  p.tagged = reinterpret_cast<uint32_t *>(ws + kChainWorkspaceHeader +
-                                          static_cast<size_t>(n_steps) * kChainLine);
+  p.done = reinterpret_cast<unsigned *>(ws + kChainDoneOffset);
+  p.tagged = reinterpret_cast<uint32_t *>(ws + kChainWorkspaceHeader);
   p.status = ctx.status;
   p.n_steps = n_steps;
   p.ctas = plan.ctas;

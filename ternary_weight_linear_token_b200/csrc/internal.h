@@ -103,12 +103,12 @@ constexpr int kChainMaxSteps = 256;
 constexpr int kStepRelu2 = 1;
 constexpr int kStepNormIn = 2;
 constexpr int kChainMaxCtas = 256;              // CTAs of one chain launch, at most
-// Workspace: the launch counter at byte 0; after the 256-byte header one
-// 128-byte line per step holding its arrival counter; then for every step
-// but the last the tagged words of the part of its output the next step
-// reads (its K values), each step's run a whole number of 128-byte lines.
+// Workspace: the launch counter at byte 0, the done counter at byte 128,
+// then for every step but the last the tagged words of the part of its
+// output the next step reads (its K values), each step's run a whole number
+// of 128-byte lines.
 constexpr size_t kChainWorkspaceHeader = 256;
-constexpr size_t kChainLine = 128;
+constexpr size_t kChainDoneOffset = 128;
 inline int64_t chain_tag_words(int64_t k_next) { return (k_next + 31) / 32 * 32; }
 struct ChainStep {
   const uint8_t *packed;

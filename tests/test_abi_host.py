@@ -177,15 +177,13 @@ def test_decode_chain_rejects_bad_arguments(tw):
 def test_decode_chain_workspace_size(tw):
     f = tw.lib.bitnet_decode_chain_workspace_size
     layer = [(3840, 2560), (2560, 2560), (6912, 2560), (2560, 6912)]
-    # 256-byte header (the launch counter); one 128-byte line per step for
-    # its arrival counter; then, for every step but the last, one 4-byte
-    # tagged word per value the next step reads
-    assert f(chain(tw, layer), 4) == 256 + 4 * 128 + 4 * (2560 + 2560 + 6912)
-    assert f(chain(tw, [(333, 64)]), 1) == 512
-    assert f(chain(tw, [(333, 64), (64, 320)]), 2) == 256 + 2 * 128 + 4 * 320
+    # 256-byte header (the launch and done counters); then, for every step
+    # but the last, one 4-byte tagged word per value the next step reads
+    assert f(chain(tw, layer), 4) == 256 + 4 * (2560 + 2560 + 6912)
+    assert f(chain(tw, [(333, 64)]), 1) == 256
+    assert f(chain(tw, [(333, 64), (64, 320)]), 2) == 256 + 4 * 320
     assert f(chain(tw, [(64, 40)]), 1) == 0          # invalid descriptors
-    assert f(chain(tw, layer * 30), 120) == (
-        256 + 120 * 128 + 4 * (30 * (2560 + 2560 + 6912 + 2560) - 2560))
+    assert f(chain(tw, layer * 30), 120) == 256 + 4 * (30 * (2560 + 2560 + 6912 + 2560) - 2560)
 
 
 def test_rms_norm_matmul_rejects_bad_arguments(tw):

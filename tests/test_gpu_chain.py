@@ -84,7 +84,9 @@ SHAPES_A = [(333, 256, True, False),     # odd N: the last exchange word holds o
             (5000, 960, True, False),    # wide: ~34 rows per CTA
             (64, 4992, False, True),     # fewer rows than CTAs
             (8192, 64, True, False),     # the largest K the next step may use
-            (160, 8192, False, True)]    # K = 8192
+            (160, 8192, False, True),    # K = 8192
+            (304, 64, True, False)]      # 2 or 4 rows of 4 packed words per CTA: a row's
+                                         # pieces fewer than the warps between them
 SHAPES_B = [(3840, 2560, False, False), (2560, 2560, False, False), (6912, 2560, True, False),
             (2560, 6912, False, False), (1, 2560, False, True)]  # one output row
 
@@ -160,19 +162,18 @@ def test_decode_chain_matches_per_launch_chain(tw):
 
 def test_decode_chain_bounded_wait_reports_timeout(tw):
     """A wait that never completes gives up (about 2 s) and is reported, with
-    no fault: the last step's arrival counter in a zero-filled workspace
-    starts at 2^30, so it never equals the count CTA 0 waits for at the end
-    (the number of CTAs), and only grows, so that count never appears.  (A
-    start below the awaited count would not do: the count could pass through
-    it.)  Only CTA 0 waits on the last step's counter; every link is
-    computed before that and is still right, the device status is
-    BITNET_ERR_TIMEOUT, and the launch counter is not advanced (zero the
-    workspace again after a timeout, as the header says)."""
+    no fault: the done counter in a zero-filled workspace starts at 2^30, so
+    it never equals the count CTA 0 waits for at the end (the number of
+    CTAs), and only grows, so that count never appears.  (A start below the
+    awaited count would not do: the count could pass through it.)  Only CTA
+    0 waits on that counter; every link is computed before that and is still
+    right, the device status is BITNET_ERR_TIMEOUT, and the launch counter
+    is not advanced (zero the workspace again after a timeout, as the header
+    says)."""
     steps, Ws = build_chain(tw, SHAPES_A[:2], 31)
     arr = tw.bitnet_decode_chain_steps(steps)
     ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
-    last = len(steps) - 1
-    ws.view(torch.int32)[(256 + 128 * last) // 4] = 1 << 30  # the last step's arrival counter
+    ws.view(torch.int32)[128 // 4] = 1 << 30  # the done counter
     assert tw.bitnet_get_device_status() == tw.OK
     x0 = x0_bits(SHAPES_A[0][1], 7)
     tw.bitnet_decode_chain(arr, bf16_t(x0), ws)
