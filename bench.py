@@ -380,7 +380,10 @@ def make_chain(tw, torch, dev, l2_bytes, layers=30, persistent=False):
                 "mode": ("one persistent launch per token (bitnet_decode_chain)" if persistent
                          else "one launch per projection and per normalisation"),
                 "timing": "CUDA graph of the timed steps"},
-        kernel_key=None, kernel_files=[], e2e_inputs=lambda: (x0["x_bits"].view(np.int16), 5120, 5120),
+        kernel_key="chain_persistent_30layers" if persistent and layers == 30 else None,
+        kernel_files=(["ternary_weight_linear_token_b200/csrc/chain.cu",
+                       "ternary_weight_linear_token_b200/csrc/common.cuh"] if persistent else []),
+        e2e_inputs=lambda: (x0["x_bits"].view(np.int16), 5120, 5120),
     )
 
 
