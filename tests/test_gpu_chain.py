@@ -160,6 +160,28 @@ def test_decode_chain_matches_per_launch_chain(tw):
     assert tw.bitnet_get_device_status() == tw.OK
 
 
+def test_decode_chain_launch_tag_wraps(tw):
+    """The 16-bit tag of launch T is (T mod 65535) + 1: with the launch
+    counter pre-set just below a multiple of 65535 the tags run 65535, 1, 2,
+    each launch's values are told apart from the previous launch's, and the
+    zero-filled tagged words (tag 0) are never taken for values."""
+    steps, Ws = build_chain(tw, SHAPES_A[:3], 41)
+    arr = tw.bitnet_decode_chain_steps(steps)
+    ws = torch.zeros(tw.bitnet_decode_chain_workspace_size(arr), dtype=torch.uint8, device=DEV)
+    ws.view(torch.int32)[0] = 65533          # the launch counter: next launch is T = 65534
+    done = 65533 * torch.cuda.get_device_properties(DEV).multi_processor_count
+    ws.view(torch.int32)[128 // 4] = done     # the done counter of those launches
+    for launch in range(3):
+        x0 = x0_bits(SHAPES_A[0][1], 500 + launch)
+        for st in steps:
+            st["Y"].fill_(float("nan"))
+        tw.bitnet_decode_chain(arr, bf16_t(x0), ws)
+        torch.cuda.synchronize()
+        check_links(steps, Ws, x0)
+        assert int(ws.view(torch.int32)[0].item()) == 65534 + launch
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
 def test_decode_chain_bounded_wait_reports_timeout(tw):
     """A wait that never completes gives up (about 2 s) and is reported, with
     no fault: the done counter in a zero-filled workspace starts at 2^30, so
