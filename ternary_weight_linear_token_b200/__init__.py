@@ -13,6 +13,7 @@ ternary_weight_linear_token_b200.build``).
 from __future__ import annotations
 
 import ctypes as C
+import functools
 import os
 
 import torch
@@ -174,9 +175,16 @@ def bitnet_quantize_act(X: torch.Tensor, xq: torch.Tensor | None = None,
 
 
 # ---------------------------------------------------------------- matmul
-def bitnet_w158a8_matmul_workspace_size(M: int, N: int, K: int, x_dtype) -> int:
-    xd = _DTYPE[x_dtype] if isinstance(x_dtype, torch.dtype) else int(x_dtype)
+@functools.lru_cache(maxsize=256)
+def _workspace_size(M: int, N: int, K: int, xd: int) -> int:
     return lib.bitnet_w158a8_matmul_workspace_size(M, N, K, xd)
+
+
+def bitnet_w158a8_matmul_workspace_size(M: int, N: int, K: int, x_dtype) -> int:
+    # a pure function of its arguments: remembered, so that a call per forward costs no
+    # second trip through ctypes
+    xd = _DTYPE[x_dtype] if isinstance(x_dtype, torch.dtype) else int(x_dtype)
+    return _workspace_size(int(M), int(N), int(K), xd)
 
 
 def bitnet_w158a8_matmul_path(M: int, N: int, K: int, x_dtype) -> int:
