@@ -239,11 +239,13 @@ def make_decode(tw, torch, dev, l2_bytes, table_lookup=False):
         kernel_files=["ternary_weight_linear_token_b200/csrc/gemv_rows.cu",
                       "ternary_weight_linear_token_b200/csrc/common.cuh"],
         e2e_inputs=lambda: (d["x_bits"].view(np.int16), 2 * d["K"], 2 * d["N"]),
-        # end to end: one host-to-host call per step (the table-lookup comparison
-        # goes through the device entry point, the host one takes no flags)
-        e2e_host=None if table_lookup else (
-            lambda i, xh, yh, stream=None: tw.bitnet_w158a8_matmul_host(
-                xh, views[i % R], gamma, X, Y, yh, weights_static=True, stream=stream)),
+        # end to end: one host-to-host call per step, through a plan per weight copy
+        # (the table-lookup comparison goes through the device entry point, the host
+        # one takes no flags)
+        e2e_plans=None if table_lookup else (
+            lambda xh, yh, stream=None: [tw.HostMatmulPlan(xh, v, gamma, X, Y, yh,
+                                                           weights_static=True, stream=stream)
+                                         for v in views]),
     )
 
 
@@ -334,10 +336,10 @@ def make_prefill(tw, torch, dev, l2_bytes, prep_in_kernel=False):
     ops = 2 * M * N * K
     return dict(
         step=step, kernel_step=kernel_step, e2e_step=lambda i, stream=None: step(0, stream),
-        e2e_host=None if prep_in_kernel else (
-            lambda i, xh, yh, stream=None: tw.bitnet_w158a8_matmul_host(
-                xh, Ps[0], gamma, Xs[0], Ys[0], yh, workspace=wss[0],
-                weights_static=True, stream=stream)),
+        e2e_plans=None if prep_in_kernel else (
+            lambda xh, yh, stream=None: [tw.HostMatmulPlan(xh, Ps[0], gamma, Xs[0], Ys[0], yh,
+                                                           workspace=wss[0], weights_static=True,
+                                                           stream=stream)]),
         units_per_step=ops, unit="TOPS",
         scale=1e-12,
         bound="tensor", launches_per_step=2, kernel_launches_per_step=1, rotate=R, X=X0,
@@ -598,22 +600,25 @@ def measure(w, tw, torch, args, dev, stream, pg, world, rank, bus):
     yh = torch.empty(w["Y"].shape, dtype=w["Y"].dtype).pin_memory()
     X = w["X"]
     e2e_step = w.get("e2e_step", w["step"])  # a step that reads X and writes Y
-    e2e_host = w.get("e2e_host")
+    e2e_plans = w.get("e2e_plans")
     # host-timed calls are short: at least 20 (and 10 untimed ones first), whatever --steps is
     n = max(20, args.e2e_steps)
     with torch.cuda.stream(stream):
-        if e2e_host is not None:
+        if e2e_plans is not None:
             # one C call per step: pinned host input -> device, the product,
-            # result -> pinned host, stream synchronised (bitnet_w158a8_matmul_host)
+            # result -> pinned host, stream synchronised (bitnet_w158a8_matmul_host,
+            # through a HostMatmulPlan per weight copy: the arguments checked once)
             xh_t = xh.view(torch.bfloat16).view(X.shape)  # the bf16 bit patterns as bf16
+            plans = e2e_plans(xh_t, yh, stream)
             for i in range(10):
-                e2e_host(i, xh_t, yh, stream)
+                plans[i % len(plans)]()
             t0 = time.perf_counter()
             for i in range(n):
-                e2e_host(i, xh_t, yh, stream)
+                plans[i % len(plans)]()
             dt = time.perf_counter() - t0
-            how = ("bitnet_w158a8_matmul_host every step: pinned host activations copied in, the "
-                   "product, the bf16 result copied back to pinned host memory, stream synchronised")
+            how = ("HostMatmulPlan (bitnet_w158a8_matmul_host over fixed buffers, arguments "
+                   "checked once) every step: pinned host activations copied in, the product, the "
+                   "bf16 result copied back to pinned host memory, stream synchronised")
         else:
             for i in range(3):
                 X.view(torch.int16).copy_(xh.view(X.shape), non_blocking=True)

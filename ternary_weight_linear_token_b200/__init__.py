@@ -235,13 +235,10 @@ def bitnet_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Ten
     return Y
 
 
-def bitnet_w158a8_matmul_host(X_host: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
-                              X_dev: torch.Tensor, Y_dev: torch.Tensor, Y_host: torch.Tensor,
-                              relu2: bool = False, workspace: torch.Tensor | None = None,
-                              weights_static: bool = False, stream=None) -> torch.Tensor:
-    """Y_host = BitLinear(X_host) in one C call: X_host (CPU, fp32/bf16, best
-    pinned) is copied to X_dev, the product writes Y_dev, which is copied to
-    Y_host (CPU, pinned); returns once Y_host holds the result."""
+def _host_call_args(X_host, packed, gamma, X_dev, Y_dev, Y_host, relu2, workspace,
+                    weights_static, stream):
+    """Checks the arguments of bitnet_w158a8_matmul_host and returns them as
+    the C call takes them (plus the workspace tensor, kept alive by the caller)."""
     if X_host.is_cuda or Y_host.is_cuda:
         raise ValueError("X_host and Y_host must be host (CPU) tensors")
     if not (X_host.is_contiguous() and Y_host.is_contiguous()):
@@ -258,13 +255,48 @@ def bitnet_w158a8_matmul_host(X_host: torch.Tensor, packed: torch.Tensor, gamma:
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=X_dev.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.bitnet_w158a8_matmul_host(_ptr(X_host), _DTYPE[X_host.dtype], _ptr(X_dev), _ptr(packed),
-                                       _ptr(gamma), M, N, K, EPI_RELU2 if relu2 else EPI_NONE,
-                                       _ptr(Y_dev), _ptr(Y_host), _DTYPE[Y_host.dtype],
-                                       _ptr(workspace), ws_bytes,
-                                       FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
-    _check(st, "bitnet_w158a8_matmul_host")
+    args = (_ptr(X_host), _DTYPE[X_host.dtype], _ptr(X_dev), _ptr(packed), _ptr(gamma), M, N, K,
+            EPI_RELU2 if relu2 else EPI_NONE, _ptr(Y_dev), _ptr(Y_host), _DTYPE[Y_host.dtype],
+            _ptr(workspace), ws_bytes, FLAG_WEIGHTS_STATIC if weights_static else 0, _stream(stream))
+    return args, workspace
+
+
+def bitnet_w158a8_matmul_host(X_host: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                              X_dev: torch.Tensor, Y_dev: torch.Tensor, Y_host: torch.Tensor,
+                              relu2: bool = False, workspace: torch.Tensor | None = None,
+                              weights_static: bool = False, stream=None) -> torch.Tensor:
+    """Y_host = BitLinear(X_host) in one C call: X_host (CPU, fp32/bf16, best
+    pinned) is copied to X_dev, the product writes Y_dev, which is copied to
+    Y_host (CPU, pinned); returns once Y_host holds the result."""
+    args, _ws = _host_call_args(X_host, packed, gamma, X_dev, Y_dev, Y_host, relu2, workspace,
+                                weights_static, stream)
+    _check(lib.bitnet_w158a8_matmul_host(*args), "bitnet_w158a8_matmul_host")
     return Y_host
+
+
+class HostMatmulPlan:
+    """bitnet_w158a8_matmul_host over fixed buffers, for a projection that
+    runs again and again (a decode loop): the arguments are checked once,
+    here; each call is then the one C call (copy X_host in, the product, copy
+    the result to Y_host, wait for the stream) with nothing else around it.
+    The caller refills X_host before a call and reads Y_host after it; the
+    tensors must stay alive and in place as long as the plan is used."""
+
+    def __init__(self, X_host: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                 X_dev: torch.Tensor, Y_dev: torch.Tensor, Y_host: torch.Tensor,
+                 relu2: bool = False, workspace: torch.Tensor | None = None,
+                 weights_static: bool = False, stream=None):
+        self._args, self._ws = _host_call_args(X_host, packed, gamma, X_dev, Y_dev, Y_host, relu2,
+                                               workspace, weights_static, stream)
+        self._keep = (X_host, packed, gamma, X_dev, Y_dev, Y_host)
+        self.Y_host = Y_host
+        self._fn = lib.bitnet_w158a8_matmul_host
+
+    def __call__(self) -> torch.Tensor:
+        st = self._fn(*self._args)
+        if st != OK:
+            raise BitnetError(st, "bitnet_w158a8_matmul_host")
+        return self.Y_host
 
 
 def bitnet_rms_norm_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,

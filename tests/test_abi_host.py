@@ -274,3 +274,19 @@ def test_host_entry_point_checks(tw):
     assert call(flags=16) == tw.ERR_INVALID_ARG
     assert call(M=4096, N=6912, K=2560) == tw.ERR_WORKSPACE
     assert call(M=0) == tw.OK
+
+
+def test_binding_refuses_host_tensors_for_device_buffers(tw):
+    """The Python binding (and the host-to-host plan) refuse CPU tensors where
+    device buffers belong, before any C call: there is no CPU fallback."""
+    import torch
+    x = torch.zeros(1, 64, dtype=torch.bfloat16)
+    y = torch.zeros(1, 16, dtype=torch.bfloat16)
+    packed = torch.zeros(16, 16, dtype=torch.uint8)
+    gamma = torch.ones(1, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tw.bitnet_w158a8_matmul(x, packed, gamma)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tw.bitnet_w158a8_matmul_host(x, packed, gamma, x.clone(), y.clone(), y)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tw.HostMatmulPlan(x, packed, gamma, x.clone(), y.clone(), y)
