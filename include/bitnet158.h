@@ -227,6 +227,40 @@ bitnet_status bitnet_w158a8_matmul_host(const void *X_host, bitnet_dtype x_dtype
                                         bitnet_stream_t stream);
 
 /* ----------------------------------------------------------------------
+ * The same host-to-host call, over fixed buffers, as a plan: for a
+ * projection that runs again and again with the same buffers (a decode
+ * loop), bitnet_host_plan_create checks the arguments once and records the
+ * copy in, the product's kernels and the copy out as one CUDA graph (it runs
+ * nothing); bitnet_host_plan_run launches that graph on `stream` and
+ * returns once Y_host holds the result (it synchronises `stream`), one
+ * submission instead of three.  The caller refills X_host before a run and
+ * reads Y_host after it.
+ *   Arguments as bitnet_w158a8_matmul_host, plus:
+ *   X_host, Y_host  page-locked host memory (cudaHostAlloc /
+ *            cudaHostRegister), else BITNET_ERR_INVALID_ARG.
+ *   plan     receives the plan (NULL on error).  Caller-owned: free it with
+ *            bitnet_host_plan_destroy.  Every buffer, the weights and the
+ *            stream must stay valid and in place while the plan is used;
+ *            run it on the device that was current at creation.
+ * Errors: those of bitnet_w158a8_matmul_host; BITNET_ERR_INVALID_ARG for a
+ * null `plan`, an empty call (M or N = 0) or pageable host memory;
+ * BITNET_ERR_CUDA when capturing or instantiating the graph fails.
+ * bitnet_host_plan_run: BITNET_ERR_INVALID_ARG for a null plan,
+ * BITNET_ERR_CUDA when the launch or the synchronisation fails.
+ * ---------------------------------------------------------------------- */
+typedef struct bitnet_host_plan_s *bitnet_host_plan;
+
+bitnet_status bitnet_host_plan_create(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                                      const uint8_t *packed, const float *gamma, int64_t M,
+                                      int64_t N, int64_t K, bitnet_epilogue epi, void *Y_dev,
+                                      void *Y_host, bitnet_dtype y_dtype, void *workspace,
+                                      size_t workspace_bytes, uint32_t flags,
+                                      bitnet_stream_t stream, bitnet_host_plan *plan);
+bitnet_status bitnet_host_plan_run(bitnet_host_plan plan);
+/* Frees the plan (NULL: nothing).  Not while a run of it is in flight. */
+void bitnet_host_plan_destroy(bitnet_host_plan plan);
+
+/* ----------------------------------------------------------------------
  * Which kernel path bitnet_w158a8_matmul takes for these sizes on the
  * current device (the paths are listed in the comment above).  Pure host
  * logic, except that the tensor-core path also needs the driver's

@@ -66,6 +66,10 @@ _SIGS = {
                                        _SZ, C.c_uint32, _P], _ST),
     "bitnet_w158a8_matmul_noalloc": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _ST,
                                       C.c_uint32, _P], _ST),
+    "bitnet_host_plan_create": ([_P, _ST, _P, _P, _P, _I64, _I64, _I64, _ST, _P, _P, _ST, _P, _SZ,
+                                 C.c_uint32, _P, C.POINTER(_P)], _ST),
+    "bitnet_host_plan_run": ([_P], _ST),
+    "bitnet_host_plan_destroy": ([_P], None),
 }
 
 
@@ -277,8 +281,10 @@ def bitnet_w158a8_matmul_host(X_host: torch.Tensor, packed: torch.Tensor, gamma:
 class HostMatmulPlan:
     """bitnet_w158a8_matmul_host over fixed buffers, for a projection that
     runs again and again (a decode loop): the arguments are checked once,
-    here; each call is then the one C call (copy X_host in, the product, copy
-    the result to Y_host, wait for the stream) with nothing else around it.
+    here, and with page-locked X_host and Y_host the copy in, the product and
+    the copy out are recorded once as a CUDA graph (bitnet_host_plan_create);
+    each call then launches it and waits (bitnet_host_plan_run).  With
+    pageable host buffers each call is the one bitnet_w158a8_matmul_host call.
     The caller refills X_host before a call and reads Y_host after it; the
     tensors must stay alive and in place as long as the plan is used."""
 
@@ -286,17 +292,38 @@ class HostMatmulPlan:
                  X_dev: torch.Tensor, Y_dev: torch.Tensor, Y_host: torch.Tensor,
                  relu2: bool = False, workspace: torch.Tensor | None = None,
                  weights_static: bool = False, stream=None):
+        self._plan = None
         self._args, self._ws = _host_call_args(X_host, packed, gamma, X_dev, Y_dev, Y_host, relu2,
                                                workspace, weights_static, stream)
         self._keep = (X_host, packed, gamma, X_dev, Y_dev, Y_host)
         self.Y_host = Y_host
-        self._fn = lib.bitnet_w158a8_matmul_host
+        self.graph = False
+        if X_host.is_pinned() and Y_host.is_pinned():
+            h = _P()
+            _check(lib.bitnet_host_plan_create(*self._args, C.byref(h)), "bitnet_host_plan_create")
+            self._plan = h
+            self.graph = True
+        self._run = lib.bitnet_host_plan_run
+        self._call = lib.bitnet_w158a8_matmul_host
 
     def __call__(self) -> torch.Tensor:
-        st = self._fn(*self._args)
+        st = self._run(self._plan) if self._plan is not None else self._call(*self._args)
         if st != OK:
-            raise BitnetError(st, "bitnet_w158a8_matmul_host")
+            raise BitnetError(st, "bitnet_host_plan_run" if self._plan is not None
+                              else "bitnet_w158a8_matmul_host")
         return self.Y_host
+
+    def close(self) -> None:
+        """Frees the CUDA graph (also done when the plan is collected)."""
+        if self._plan is not None:
+            lib.bitnet_host_plan_destroy(self._plan)
+            self._plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def bitnet_rms_norm_w158a8_matmul(X: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,

@@ -285,6 +285,55 @@ int matmul_args_status(const void *X, int x_dtype, const float *s, const uint8_t
 
 using namespace bitnet;
 
+namespace {
+
+// The argument checks of bitnet_w158a8_matmul_host (also those of a plan).
+bitnet_status check_host_call(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                              const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
+                              int64_t K, bitnet_epilogue epi, void *Y_dev, void *Y_host,
+                              bitnet_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                              uint32_t flags) {
+  if (x_dtype == BITNET_I8) return BITNET_ERR_INVALID_ARG;
+  if (bitnet_status st = check_matmul(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, epi, Y_dev,
+                                      y_dtype, workspace, workspace_bytes, flags, false))
+    return st;
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (X_host == nullptr || Y_host == nullptr) return BITNET_ERR_INVALID_ARG;
+  return BITNET_OK;
+}
+
+// Copy in, the product, copy out, all on ctx.stream (no wait).
+bitnet_status enqueue_host_call(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                                const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
+                                int64_t K, bitnet_epilogue epi, void *Y_dev, void *Y_host,
+                                bitnet_dtype y_dtype, void *workspace, uint32_t flags,
+                                const LaunchCtx &ctx) {
+  const size_t x_bytes = static_cast<size_t>(M) * K * elem_size(x_dtype);
+  const size_t y_bytes = static_cast<size_t>(M) * N * elem_size(y_dtype);
+  if (cudaMemcpyAsync(X_dev, X_host, x_bytes, cudaMemcpyHostToDevice, ctx.stream) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  const bool relu2 = epi == BITNET_EPI_RELU2, wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
+  const bitnet_status st =
+      (flags & BITNET_FLAG_TABLE_LOOKUP) != 0
+          ? from_cuda(launch_lut(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y_dev,
+                                 y_dtype, wstatic, ctx))
+          : run_matmul(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y_dev, y_dtype,
+                       workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0,
+                       (flags & BITNET_FLAG_PREP_IN_KERNEL) != 0, ctx);
+  if (st != BITNET_OK) return st;
+  if (cudaMemcpyAsync(Y_host, Y_dev, y_bytes, cudaMemcpyDeviceToHost, ctx.stream) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  return BITNET_OK;
+}
+
+}  // namespace
+
+// A host-to-host call captured once as a CUDA graph.
+struct bitnet_host_plan_s {
+  cudaGraphExec_t exec;
+  cudaStream_t stream;
+};
+
 extern "C" {
 
 int bitnet_version(void) { return 10000; }
@@ -353,30 +402,82 @@ bitnet_status bitnet_w158a8_matmul_host(const void *X_host, bitnet_dtype x_dtype
                                         void *Y_host, bitnet_dtype y_dtype, void *workspace,
                                         size_t workspace_bytes, uint32_t flags,
                                         bitnet_stream_t stream) {
-  if (x_dtype == BITNET_I8) return BITNET_ERR_INVALID_ARG;
-  if (bitnet_status st = check_matmul(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, epi, Y_dev,
-                                      y_dtype, workspace, workspace_bytes, flags, false))
+  if (bitnet_status st = check_host_call(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi, Y_dev,
+                                         Y_host, y_dtype, workspace, workspace_bytes, flags))
     return st;
   if (M == 0 || N == 0) return BITNET_OK;
-  if (X_host == nullptr || Y_host == nullptr) return BITNET_ERR_INVALID_ARG;
   LaunchCtx ctx;
   if (bitnet_status st = device_ctx(stream, &ctx)) return st;
-  const size_t x_bytes = static_cast<size_t>(M) * K * elem_size(x_dtype);
-  const size_t y_bytes = static_cast<size_t>(M) * N * elem_size(y_dtype);
-  if (cudaMemcpyAsync(X_dev, X_host, x_bytes, cudaMemcpyHostToDevice, ctx.stream) != cudaSuccess)
-    return BITNET_ERR_CUDA;
-  const bool relu2 = epi == BITNET_EPI_RELU2, wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
-  const bitnet_status st =
-      (flags & BITNET_FLAG_TABLE_LOOKUP) != 0
-          ? from_cuda(launch_lut(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y_dev,
-                                 y_dtype, wstatic, ctx))
-          : run_matmul(X_dev, x_dtype, nullptr, packed, gamma, M, N, K, relu2, Y_dev, y_dtype,
-                       workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0,
-                       (flags & BITNET_FLAG_PREP_IN_KERNEL) != 0, ctx);
-  if (st != BITNET_OK) return st;
-  if (cudaMemcpyAsync(Y_host, Y_dev, y_bytes, cudaMemcpyDeviceToHost, ctx.stream) != cudaSuccess)
-    return BITNET_ERR_CUDA;
+  if (bitnet_status st = enqueue_host_call(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi,
+                                           Y_dev, Y_host, y_dtype, workspace, flags, ctx))
+    return st;
   return cudaStreamSynchronize(ctx.stream) == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+bitnet_status bitnet_host_plan_create(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                                      const uint8_t *packed, const float *gamma, int64_t M,
+                                      int64_t N, int64_t K, bitnet_epilogue epi, void *Y_dev,
+                                      void *Y_host, bitnet_dtype y_dtype, void *workspace,
+                                      size_t workspace_bytes, uint32_t flags,
+                                      bitnet_stream_t stream, bitnet_host_plan *plan) {
+  if (plan == nullptr) return BITNET_ERR_INVALID_ARG;
+  *plan = nullptr;
+  if (bitnet_status st = check_host_call(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi, Y_dev,
+                                         Y_host, y_dtype, workspace, workspace_bytes, flags))
+    return st;
+  if (M == 0 || N == 0) return BITNET_ERR_INVALID_ARG;
+  // the graph's copies need page-locked host memory
+  for (const void *h : {X_host, static_cast<const void *>(Y_host)}) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, h) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return BITNET_ERR_INVALID_ARG;
+    }
+    if (a.type != cudaMemoryTypeHost) return BITNET_ERR_INVALID_ARG;
+  }
+  LaunchCtx ctx;
+  if (bitnet_status st = device_ctx(stream, &ctx)) return st;
+  // Captured on a stream of its own (the caller's may be the legacy default
+  // stream, which cannot be captured), launched later on the caller's.
+  cudaStream_t cap = nullptr;
+  if (cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking) != cudaSuccess) return BITNET_ERR_CUDA;
+  LaunchCtx cctx = ctx;
+  cctx.stream = cap;
+  cudaGraph_t graph = nullptr;
+  bitnet_status st = BITNET_OK;
+  if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    st = BITNET_ERR_CUDA;
+  } else {
+    st = enqueue_host_call(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi, Y_dev, Y_host,
+                           y_dtype, workspace, flags, cctx);
+    // always end the capture, also after a failed enqueue
+    if (cudaStreamEndCapture(cap, &graph) != cudaSuccess && st == BITNET_OK) st = BITNET_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  if (st == BITNET_OK &&
+      (graph == nullptr || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess))
+    st = BITNET_ERR_CUDA;
+  if (graph != nullptr) cudaGraphDestroy(graph);
+  cudaStreamDestroy(cap);
+  if (st != BITNET_OK) {
+    (void)cudaGetLastError();
+    if (exec != nullptr) cudaGraphExecDestroy(exec);
+    return st;
+  }
+  *plan = new bitnet_host_plan_s{exec, ctx.stream};
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_host_plan_run(bitnet_host_plan plan) {
+  if (plan == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (cudaGraphLaunch(plan->exec, plan->stream) != cudaSuccess) return BITNET_ERR_CUDA;
+  return cudaStreamSynchronize(plan->stream) == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+void bitnet_host_plan_destroy(bitnet_host_plan plan) {
+  if (plan == nullptr) return;
+  cudaGraphExecDestroy(plan->exec);
+  delete plan;
 }
 
 bitnet_path bitnet_w158a8_matmul_path(int64_t M, int64_t N, int64_t K, bitnet_dtype x_dtype) {

@@ -276,6 +276,32 @@ def test_host_entry_point_checks(tw):
     assert call(M=0) == tw.OK
 
 
+def test_host_plan_checks(tw):
+    """A plan takes the host entry point's checks, all before any CUDA call,
+    and refuses a null plan pointer and an empty call; running or freeing a
+    null plan is safe."""
+    f = tw.lib.bitnet_host_plan_create
+    H = C.c_void_p(0x7000000)
+
+    def create(Xh=H, xd=1, Xd=A, M=1, N=8, K=64, Yd=Cc, Yh=H, flags=0, out=True):
+        h = C.c_void_p(0x1234)
+        st = f(Xh, xd, Xd, B, G, M, N, K, 0, Yd, Yh, 1, None, 0, flags, None,
+               C.byref(h) if out else None)
+        if out:
+            assert h.value is None  # NULL on every error
+        return st
+
+    assert create(out=False) == tw.ERR_INVALID_ARG
+    assert create(Xh=None) == tw.ERR_INVALID_ARG
+    assert create(xd=2) == tw.ERR_INVALID_ARG
+    assert create(Xd=MIS) == tw.ERR_MISALIGNED
+    assert create(K=40) == tw.ERR_UNSUPPORTED_SHAPE
+    assert create(flags=16) == tw.ERR_INVALID_ARG
+    assert create(M=0) == tw.ERR_INVALID_ARG
+    assert tw.lib.bitnet_host_plan_run(None) == tw.ERR_INVALID_ARG
+    tw.lib.bitnet_host_plan_destroy(None)
+
+
 def test_binding_refuses_host_tensors_for_device_buffers(tw):
     """The Python binding (and the host-to-host plan) refuse CPU tensors where
     device buffers belong, before any C call: there is no CPU fallback."""

@@ -568,6 +568,7 @@ def test_host_entry_point(tw, M, N, K, dt):
         assert np.array_equal(Yh.view(torch.int16).numpy().view(np.uint16), ref.to_bf16(want_o))
     # the same call through a plan (arguments checked once), with the host input refilled
     plan = tw.HostMatmulPlan(Xh, pd, gd, X2, Y2, Yh, weights_static=True)
+    assert plan.graph  # page-locked buffers: recorded once as a CUDA graph
     for r in range(2):
         x2 = rng.standard_t(3, (M, K)).astype(np.float32)
         Xd2, xexact2 = as_x(x2, dt)
@@ -577,6 +578,7 @@ def test_host_entry_point(tw, M, N, K, dt):
         want2 = ref.bitlinear(xexact2, po, go, N)["y"]
         got2 = Yh.numpy() if dt == "f32" else Yh.view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(got2, want2 if dt == "f32" else ref.to_bf16(want2)), r
+    plan.close()
     assert tw.bitnet_get_device_status() == tw.OK
 
 
