@@ -310,8 +310,12 @@ bitnet_status enqueue_host_call(const void *X_host, bitnet_dtype x_dtype, void *
                                 const LaunchCtx &ctx) {
   const size_t x_bytes = static_cast<size_t>(M) * K * elem_size(x_dtype);
   const size_t y_bytes = static_cast<size_t>(M) * N * elem_size(y_dtype);
-  if (cudaMemcpyAsync(X_dev, X_host, x_bytes, cudaMemcpyHostToDevice, ctx.stream) != cudaSuccess)
-    return BITNET_ERR_CUDA;
+  // a few KB (decode): a copy kernel chained to the product; more: the copy engine
+  const cudaError_t in =
+      small_copy_ok(X_host, X_dev, x_bytes)
+          ? launch_small_copy(X_host, X_dev, x_bytes, ctx)
+          : cudaMemcpyAsync(X_dev, X_host, x_bytes, cudaMemcpyHostToDevice, ctx.stream);
+  if (in != cudaSuccess) return BITNET_ERR_CUDA;
   const bool relu2 = epi == BITNET_EPI_RELU2, wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
   const bitnet_status st =
       (flags & BITNET_FLAG_TABLE_LOOKUP) != 0
@@ -321,9 +325,11 @@ bitnet_status enqueue_host_call(const void *X_host, bitnet_dtype x_dtype, void *
                        workspace, wstatic, (flags & BITNET_FLAG_WEIGHTS_EXPANDED) != 0,
                        (flags & BITNET_FLAG_PREP_IN_KERNEL) != 0, ctx);
   if (st != BITNET_OK) return st;
-  if (cudaMemcpyAsync(Y_host, Y_dev, y_bytes, cudaMemcpyDeviceToHost, ctx.stream) != cudaSuccess)
-    return BITNET_ERR_CUDA;
-  return BITNET_OK;
+  const cudaError_t out =
+      small_copy_ok(Y_host, Y_dev, y_bytes)
+          ? launch_small_copy(Y_dev, Y_host, y_bytes, ctx)
+          : cudaMemcpyAsync(Y_host, Y_dev, y_bytes, cudaMemcpyDeviceToHost, ctx.stream);
+  return out == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
 }  // namespace

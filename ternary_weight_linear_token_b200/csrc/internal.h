@@ -97,6 +97,14 @@ cudaError_t launch_prefill(const int8_t *xq, const float *s, const int8_t *w8,
                            void *Y, int y_kind, const LaunchCtx &ctx,
                            const PrefillPrep *prep = nullptr);
 
+// host_copy.cu: small copies between page-locked host memory and the device
+// by a kernel (16-byte pieces, programmatic dependent launch).  small_copy_ok:
+// bytes <= kSmallCopyMax, a multiple of 16, both pointers 16-byte aligned and
+// `host` page-locked memory the device addresses at the same address.
+constexpr size_t kSmallCopyMax = 64 * 1024;
+bool small_copy_ok(const void *host, const void *dev, size_t bytes);
+cudaError_t launch_small_copy(const void *src, void *dst, size_t bytes, const LaunchCtx &ctx);
+
 // chain.cu: persistent M = 1 chain of BitLinear projections (one
 // cooperative launch).  Step flags mirror BITNET_STEP_*.
 constexpr int kChainMaxSteps = 256;
