@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <new>
 
 #include "../../include/bitnet158.h"
 #include "internal.h"
@@ -470,7 +471,12 @@ bitnet_status bitnet_host_plan_create(const void *X_host, bitnet_dtype x_dtype, 
     if (exec != nullptr) cudaGraphExecDestroy(exec);
     return st;
   }
-  *plan = new bitnet_host_plan_s{exec, ctx.stream};
+  bitnet_host_plan made = new (std::nothrow) bitnet_host_plan_s{exec, ctx.stream};
+  if (made == nullptr) {  // no exception crosses the C boundary
+    cudaGraphExecDestroy(exec);
+    return BITNET_ERR_CUDA;
+  }
+  *plan = made;
   return BITNET_OK;
 }
 
