@@ -300,9 +300,12 @@ class HostMatmulPlan:
         self.graph = False
         if X_host.is_pinned() and Y_host.is_pinned():
             h = _P()
-            _check(lib.bitnet_host_plan_create(*self._args, C.byref(h)), "bitnet_host_plan_create")
-            self._plan = h
-            self.graph = True
+            st = lib.bitnet_host_plan_create(*self._args, C.byref(h))
+            if st == OK:
+                self._plan = h
+                self.graph = True
+            elif st != ERR_CUDA:  # argument errors raise; a graph that could not be
+                _check(st, "bitnet_host_plan_create")  # made leaves the per-call path
         self._run = lib.bitnet_host_plan_run
         self._call = lib.bitnet_w158a8_matmul_host
 
