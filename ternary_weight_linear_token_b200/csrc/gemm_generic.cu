@@ -26,8 +26,9 @@ __global__ void __launch_bounds__(32 * kWarps) generic_kernel(const int8_t *xq, 
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTokens;
-  if (n < N) {
+  // token blocks of kTokens, strided over gridDim.y (at most 65535 of them)
+  for (int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTokens; n < N && m0 < M;
+       m0 += static_cast<int64_t>(gridDim.y) * kTokens) {
     const float gamma = *gamma_ptr;
     const uint32_t *row = reinterpret_cast<const uint32_t *>(packed + n * (K / 4));
     const int64_t words = K / 16;
@@ -63,8 +64,9 @@ __global__ void __launch_bounds__(32 * kWarps) generic_kernel(const int8_t *xq, 
 template <int YK, bool RELU2>
 cudaError_t go(const int8_t *xq, const float *s, const uint8_t *packed, const float *gamma,
                int64_t M, int64_t N, int64_t K, void *Y, const LaunchCtx &ctx) {
+  const int64_t mblocks = ceil_div(M, kTokens);
   const dim3 grid(static_cast<unsigned>(ceil_div(N, kWarps)),
-                  static_cast<unsigned>(ceil_div(M, kTokens)));
+                  static_cast<unsigned>(mblocks < 65535 ? mblocks : 65535));
   return launch_k(generic_kernel<YK, RELU2>, grid, dim3(32 * kWarps), 0, ctx, xq, s, packed,
                   gamma, M, N, K, Y);
 }

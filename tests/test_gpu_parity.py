@@ -173,6 +173,37 @@ def test_matmul_parity(tw, M, N, K, xdtype):
     assert all(exact.values()), f"within tolerance but not bit-identical: {exact}"
 
 
+# The extremes of the accepted sizes, kept cheap for the oracle by the other
+# dimensions: K up to 2^22 (|acc| <= 127 K stays far inside int32; the
+# activations no longer fit any kernel's shared-memory window) for 1, 3, 8
+# and 40 tokens; 2^17 tokens (1024 row tiles of the tensor-core path); and
+# 1.1 M tokens on the dp4a kernel (K % 64 != 0), more token blocks than a
+# grid's y dimension holds.
+EXTREME_SHAPES = [(1, 7, 1 << 20), (3, 5, 1 << 22), (8, 9, 1 << 20), (40, 6, 1 << 20),
+                  (1 << 17, 24, 64), (100003, 3, 128), (1100000, 3, 16)]
+
+
+@pytest.mark.parametrize("M,N,K", EXTREME_SHAPES)
+def test_matmul_parity_extreme_sizes(tw, M, N, K):
+    """Every kernel path at the largest sizes the checks accept that still fit
+    a test: int32 accumulators and bf16 outputs bit-exact, bf16 input."""
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    W = synth.latent_weights(rng, N, K)
+    x = rng.standard_t(3, (M, K)).astype(np.float32)
+    packed_d, gamma_d, packed_o, gamma_o = quantize_weights_both(W)
+    assert np.array_equal(np_of(packed_d), packed_o)
+    Xd, xexact = as_x(x, "bf16")
+    xq_o, s_o = ref.quantize_act(xexact)
+    acc_o = ref.matmul_acc(xq_o, packed_o, N, K)
+    Y = tw.bitnet_w158a8_matmul(Xd, packed_d, gamma_d, out_dtype=torch.int32)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_of(Y), acc_o), "int32 accumulators differ"
+    Y = tw.bitnet_w158a8_matmul(Xd, packed_d, gamma_d, relu2=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits_of(Y), ref.to_bf16(ref.epilogue(acc_o, s_o, gamma_o, True)))
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
 PREP_SHAPES = [(33, 300, 192), (128, 256, 128), (129, 257, 2624), (300, 600, 2560),
                (256, 520, 64), (1000, 512, 2560), (640, 1100, 384), (130, 70, 208)]
 
