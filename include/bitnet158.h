@@ -229,9 +229,10 @@ bitnet_status bitnet_w158a8_matmul_host(const void *X_host, bitnet_dtype x_dtype
 /* ----------------------------------------------------------------------
  * The same host-to-host call, over fixed buffers, as a plan: for a
  * projection that runs again and again with the same buffers (a decode
- * loop), bitnet_host_plan_create checks the arguments once and records the
- * copy in, the product's kernels and the copy out as one CUDA graph (it runs
- * nothing); bitnet_host_plan_run launches that graph on `stream` and
+ * loop), bitnet_host_plan_create checks the arguments once, records the
+ * copy in, the product's kernels and the copy out as one CUDA graph and
+ * uploads it to the device (it runs nothing; the upload is enqueued on
+ * `stream`); bitnet_host_plan_run launches that graph on `stream` and
  * returns once Y_host holds the result (it synchronises `stream`), one
  * submission instead of three.  The caller refills X_host before a run and
  * reads Y_host after it.

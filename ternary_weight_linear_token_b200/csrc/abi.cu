@@ -464,6 +464,9 @@ bitnet_status bitnet_host_plan_create(const void *X_host, bitnet_dtype x_dtype, 
   if (st == BITNET_OK &&
       (graph == nullptr || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess))
     st = BITNET_ERR_CUDA;
+  // uploaded now, on the caller's stream, so that the first run costs what
+  // every later one does
+  if (st == BITNET_OK && cudaGraphUpload(exec, ctx.stream) != cudaSuccess) st = BITNET_ERR_CUDA;
   if (graph != nullptr) cudaGraphDestroy(graph);
   cudaStreamDestroy(cap);
   if (st != BITNET_OK) {
