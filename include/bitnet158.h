@@ -234,8 +234,10 @@ bitnet_status bitnet_w158a8_matmul_host(const void *X_host, bitnet_dtype x_dtype
  * uploads it to the device (it runs nothing; the upload is enqueued on
  * `stream`); bitnet_host_plan_run launches that graph on `stream` and
  * returns once Y_host holds the result (it synchronises `stream`), one
- * submission instead of three.  The caller refills X_host before a run and
- * reads Y_host after it.
+ * submission instead of three.  A large call on the tensor-core path is
+ * recorded as a pipeline of token chunks over three streams, so that the
+ * copies in and out overlap the product (same results).  The caller refills
+ * X_host before a run and reads Y_host after it.
  *   Arguments as bitnet_w158a8_matmul_host, plus:
  *   X_host, Y_host  page-locked host memory (cudaHostAlloc /
  *            cudaHostRegister), else BITNET_ERR_INVALID_ARG.

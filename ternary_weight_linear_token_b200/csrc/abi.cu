@@ -333,6 +333,99 @@ bitnet_status enqueue_host_call(const void *X_host, bitnet_dtype x_dtype, void *
   return out == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
+// The same work for a large call on the tensor-core path, as a pipeline of
+// token chunks over three streams: chunk c + 1 is copied in (stream `in`)
+// while chunk c is computed (ctx.stream) and the finished chunks are copied
+// out (stream `out`), so that the two copy directions and the product
+// overlap.  Every chunk but the last has the same number of tokens, so the
+// int8 weights the first chunk expanded into the workspace sit where the
+// next equal chunks look for them (BITNET_FLAG_WEIGHTS_EXPANDED); the last,
+// smaller chunk expands them again.  Only recorded into a plan's graph: the
+// streams and events are the capture's and are released after it.
+constexpr int64_t kPipeChunks = 8;
+constexpr int64_t kPipeMinTokens = 256;
+constexpr size_t kPipeMinBytes = size_t(4) << 20;
+
+bool pipeline_fits(bitnet_dtype x_dtype, int64_t M, int64_t N, int64_t K, bitnet_dtype y_dtype,
+                   uint32_t flags) {
+  if ((flags & ~BITNET_FLAG_WEIGHTS_STATIC) != 0) return false;
+  if (M < kPipeMinTokens || !use_prefill(M, N, K, x_dtype) || !prefill_supported(M, N, K))
+    return false;
+  return static_cast<size_t>(M) * (K * elem_size(x_dtype) + N * elem_size(y_dtype)) >=
+         kPipeMinBytes;
+}
+
+// Side streams and events of a pipelined capture, made before it and
+// released after it ends (a stream that joined a capture must not go away
+// while the capture is open).
+struct PipeRes {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t ev[2 * kPipeChunks + 3] = {};
+  bool make() {
+    if (cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess)
+      return false;
+    for (cudaEvent_t &e : ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  void release() {
+    for (cudaEvent_t &e : ev)
+      if (e != nullptr) cudaEventDestroy(e);
+    if (in != nullptr) cudaStreamDestroy(in);
+    if (out != nullptr) cudaStreamDestroy(out);
+  }
+};
+
+bitnet_status enqueue_host_pipeline(const void *X_host, bitnet_dtype x_dtype, void *X_dev,
+                                    const uint8_t *packed, const float *gamma, int64_t M,
+                                    int64_t N, int64_t K, bitnet_epilogue epi, void *Y_dev,
+                                    void *Y_host, bitnet_dtype y_dtype, void *workspace,
+                                    uint32_t flags, const PipeRes &r, const LaunchCtx &ctx) {
+  const int64_t per = ceil_div(ceil_div(M, kPipeChunks), int64_t(128)) * 128;  // whole row tiles
+  const int64_t chunks = ceil_div(M, per);  // <= kPipeChunks
+  const size_t xrow = static_cast<size_t>(K) * elem_size(x_dtype);
+  const size_t yrow = static_cast<size_t>(N) * elem_size(y_dtype);
+  // fork: both side streams join the capture after the main stream's start
+  if (cudaEventRecord(r.ev[0], ctx.stream) != cudaSuccess ||
+      cudaStreamWaitEvent(r.in, r.ev[0], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(r.out, r.ev[0], 0) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  bitnet_status st = BITNET_OK;
+  const bool relu2 = epi == BITNET_EPI_RELU2, wstatic = (flags & BITNET_FLAG_WEIGHTS_STATIC) != 0;
+  for (int64_t c = 0; st == BITNET_OK && c < chunks; ++c) {
+    const int64_t m0 = c * per, mc = M - m0 < per ? M - m0 : per;
+    uint8_t *xd = static_cast<uint8_t *>(X_dev) + static_cast<size_t>(m0) * xrow;
+    uint8_t *yd = static_cast<uint8_t *>(Y_dev) + static_cast<size_t>(m0) * yrow;
+    const cudaEvent_t in_done = r.ev[1 + 2 * c], y_done = r.ev[2 + 2 * c];
+    if (cudaMemcpyAsync(xd, static_cast<const uint8_t *>(X_host) + static_cast<size_t>(m0) * xrow,
+                        static_cast<size_t>(mc) * xrow, cudaMemcpyHostToDevice, r.in) != cudaSuccess ||
+        cudaEventRecord(in_done, r.in) != cudaSuccess ||
+        cudaStreamWaitEvent(ctx.stream, in_done, 0) != cudaSuccess) {
+      st = BITNET_ERR_CUDA;
+      break;
+    }
+    const bool reuse = c > 0 && mc == per;  // the first chunk's expansion, at the same offset
+    st = run_matmul(xd, x_dtype, nullptr, packed, gamma, mc, N, K, relu2, yd, y_dtype, workspace,
+                    wstatic, reuse, false, ctx);
+    if (st != BITNET_OK) break;
+    if (cudaEventRecord(y_done, ctx.stream) != cudaSuccess ||
+        cudaStreamWaitEvent(r.out, y_done, 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t *>(Y_host) + static_cast<size_t>(m0) * yrow, yd,
+                        static_cast<size_t>(mc) * yrow, cudaMemcpyDeviceToHost, r.out) != cudaSuccess)
+      st = BITNET_ERR_CUDA;
+  }
+  // join (also after an error, so that the capture can end): the main
+  // stream ends after both side streams
+  const cudaEvent_t join_in = r.ev[2 * kPipeChunks + 1], join_out = r.ev[2 * kPipeChunks + 2];
+  if (cudaEventRecord(join_in, r.in) != cudaSuccess ||
+      cudaStreamWaitEvent(ctx.stream, join_in, 0) != cudaSuccess ||
+      cudaEventRecord(join_out, r.out) != cudaSuccess ||
+      cudaStreamWaitEvent(ctx.stream, join_out, 0) != cudaSuccess)
+    st = BITNET_ERR_CUDA;
+  return st;
+}
+
 }  // namespace
 
 // A host-to-host call captured once as a CUDA graph.
@@ -452,14 +545,20 @@ bitnet_status bitnet_host_plan_create(const void *X_host, bitnet_dtype x_dtype, 
   cctx.stream = cap;
   cudaGraph_t graph = nullptr;
   bitnet_status st = BITNET_OK;
-  if (cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+  const bool pipe = pipeline_fits(x_dtype, M, N, K, y_dtype, flags);
+  PipeRes res;
+  if (pipe && !res.make()) st = BITNET_ERR_CUDA;
+  if (st == BITNET_OK && cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
     st = BITNET_ERR_CUDA;
-  } else {
-    st = enqueue_host_call(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi, Y_dev, Y_host,
-                           y_dtype, workspace, flags, cctx);
+  else if (st == BITNET_OK) {
+    st = pipe ? enqueue_host_pipeline(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi, Y_dev,
+                                      Y_host, y_dtype, workspace, flags, res, cctx)
+              : enqueue_host_call(X_host, x_dtype, X_dev, packed, gamma, M, N, K, epi, Y_dev,
+                                  Y_host, y_dtype, workspace, flags, cctx);
     // always end the capture, also after a failed enqueue
     if (cudaStreamEndCapture(cap, &graph) != cudaSuccess && st == BITNET_OK) st = BITNET_ERR_CUDA;
   }
+  res.release();
   cudaGraphExec_t exec = nullptr;
   if (st == BITNET_OK &&
       (graph == nullptr || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess))

@@ -572,11 +572,15 @@ def test_rms_norm_matmul(tw, M, N, K, dt, relu2):
 
 
 @pytest.mark.parametrize("M,N,K,dt", [(1, 2560, 2560, "bf16"), (8, 300, 320, "f32"),
-                                      (300, 600, 2560, "bf16")])
+                                      (300, 600, 2560, "bf16"), (1000, 1600, 2560, "bf16"),
+                                      (916, 1100, 1024, "f32")])
 def test_host_entry_point(tw, M, N, K, dt):
     """bitnet_w158a8_matmul_host (pinned host input and output, one call)
     gives exactly the device entry point's output, on the fused, mma.sync and
-    tensor-core paths, and the oracle's."""
+    tensor-core paths, and the oracle's; so does a HostMatmulPlan, whose
+    graph for the last two shapes is a pipeline of 128-token chunks (the last
+    chunk 104 tokens on the tensor-core path, or 20 tokens on the mma.sync
+    path)."""
     rng = np.random.default_rng(M + N + K)
     W = synth.latent_weights(rng, N, K)
     x = rng.standard_t(3, (M, K)).astype(np.float32)
