@@ -617,6 +617,32 @@ def test_host_entry_point(tw, M, N, K, dt):
     assert tw.bitnet_get_device_status() == tw.OK
 
 
+def test_host_plan_pageable_buffers(tw):
+    """A HostMatmulPlan over pageable host tensors records no graph and makes
+    the host entry point's call each time (the driver stages the copies);
+    the results are the oracle's."""
+    M, N, K = 1, 640, 1024
+    rng = np.random.default_rng(4242)
+    W = synth.latent_weights(rng, N, K)
+    pd, gd, po, go = quantize_weights_both(W)
+    Xh = torch.empty((M, K), dtype=torch.bfloat16)
+    Yh = torch.empty((M, N), dtype=torch.bfloat16)
+    assert not Xh.is_pinned() and not Yh.is_pinned()
+    X2 = torch.empty((M, K), dtype=torch.bfloat16, device=DEV)
+    Y2 = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    plan = tw.HostMatmulPlan(Xh, pd, gd, X2, Y2, Yh, relu2=True)
+    assert not plan.graph
+    for r in range(2):
+        x = rng.standard_t(3, (M, K)).astype(np.float32)
+        Xd, xexact = as_x(x, "bf16")
+        Xh.copy_(Xd.cpu())
+        plan()
+        want = ref.bitlinear(xexact, po, go, N, relu2=True)["y"]
+        assert np.array_equal(Yh.view(torch.int16).numpy().view(np.uint16), ref.to_bf16(want)), r
+    plan.close()
+    assert tw.bitnet_get_device_status() == tw.OK
+
+
 def test_repeatable(tw):
     d = synth.config_inputs("sweep", M=8, proj=0)
     pd, gd = tw.bitnet_quantize_weights(f32_t(d["W"]))
