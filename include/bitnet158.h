@@ -433,7 +433,10 @@ const char *bitnet_status_string(bitnet_status status);
  * (BITNET_ERR_TIMEOUT after a bounded wait gave up). */
 bitnet_status bitnet_get_device_status(bitnet_stream_t stream);
 
-/* ABI version of this header: major * 10000 + minor * 100 + patch. */
+/* ABI version of this header: major * 10000 + minor * 100 + patch.  1.1:
+ * the path query, the host-to-host call and its plans; the chain workspace
+ * holds tagged link values (its size from bitnet_decode_chain_workspace_size). */
+#define BITNET_VERSION 10100
 int bitnet_version(void);
 
 #ifdef __cplusplus

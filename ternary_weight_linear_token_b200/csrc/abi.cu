@@ -436,7 +436,7 @@ struct bitnet_host_plan_s {
 
 extern "C" {
 
-int bitnet_version(void) { return 10000; }
+int bitnet_version(void) { return BITNET_VERSION; }
 
 const char *bitnet_status_string(bitnet_status status) {
   switch (status) {

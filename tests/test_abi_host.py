@@ -43,7 +43,8 @@ def test_status_strings_and_version(tw):
     for st in range(8):
         assert isinstance(tw.status_string(st), str) and tw.status_string(st)
     assert tw.status_string(99) == "unknown status"
-    assert tw.version() == 10000
+    m = re.search(r"#define BITNET_VERSION (\d+)", open(HEADER).read())
+    assert m and tw.version() == int(m.group(1)) == 10100  # the library is the header's
 
 
 # Fake, suitably aligned device addresses: the calls below must be rejected by
