@@ -60,7 +60,7 @@ constexpr int kHeader = 1024;
 constexpr int kBarConsumers = 1;            // named barrier of the consumer warps
 constexpr int kChunks = 2;                  // 8-element input chunks per thread: K <= 8192
 constexpr int kRowsPerPass = 4;             // rows a warp carries at once in the dot products
-constexpr unsigned kFirstPollDelayNs = 300;  // before a step's first input loads
+constexpr long long kFirstPollDelayCycles = 885;  // before a step's first input loads (450 ns)
 
 __host__ __device__ constexpr int align128(int n) { return (n + 127) / 128 * 128; }
 // Shared-memory copies made once at the start: the step descriptors, every
@@ -206,12 +206,18 @@ __device__ __forceinline__ bool wait_or_stop(uint64_t *bar, uint32_t parity,
 __device__ __forceinline__ bool load_tagged(const uint32_t *src, int nchunks, int tid, uint32_t tb,
                                             float (&v)[kChunks][8], int *status) {
   uint4 t[kChunks][2];
-  // The first loads wait about 0.3 us: polling the moment the CTA is done,
+  // The first loads wait about 0.45 us: polling the moment the CTA is done,
   // while the last CTAs still store, slowed every step (30-layer stack: 575
-  // us per token without the delay, 548 / 480 / 447 / 462 / 458 with 50 /
-  // 150 / 300 / 600 / 1000 ns; sleeping only after a first poll that found
-  // missing words: 705).
-  __nanosleep(kFirstPollDelayNs);
+  // us per token without the delay; __nanosleep of 50 / 150 / 300 / 600 /
+  // 1000 ns: 548 / 480 / 447 / 462 / 458; sleeping only after a first poll
+  // that found missing words: 705).  A spin on the SM clock is exact where
+  // the sleep is not: 200 / 300 / 450 / 600 / 800 ns at 1965 MHz gave
+  // 472 / 450 / 430 / 434 / 456 us per token.
+  {
+    const long long t_start = clock64();
+    while (clock64() - t_start < kFirstPollDelayCycles) {
+    }
+  }
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
     const int c = tid + i * kCThreads;
